@@ -1,0 +1,462 @@
+"""Benchmark: fused QKV + decode attention step on a two-tier (HBM / mapped host) paged KV cache.
+
+Default workload (N=1): the Llama-3-8B-shaped layer with the whole cache in HBM — batch 16,
+hidden 4096, 32 q / 8 kv heads, head_dim 128, RoPE theta 5e5, 32768 cached tokens per
+sequence in 16-token blocks. A step is one decode step of one layer through the C ABI
+(dkv_decode_step: projection, split-K attention, combine). Inputs are synthetic (seeded
+N(0,1) activations and KV, W ~ N(0, 1/hidden)), generated on the device.
+
+Multi-GPU: every rank runs an independent replica of the workload (the step has no
+cross-GPU exchange); value = tokens of all ranks / max-over-ranks time.
+
+Prints one JSON line on rank 0. `--impl reference` times the fp64 CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as WL  # noqa: E402
+
+METRIC = "fused QKV+decode-attn tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="dkv", choices=["dkv", "reference"])
+    ap.add_argument("--config", default="8b_hbm", choices=sorted(WL.CONFIGS))
+    ap.add_argument("--attn-splits", type=int, default=0)
+    ap.add_argument("--proj-splits", type=int, default=0)
+    ap.add_argument("--host-flags", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- helpers
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def src_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "kv_cache_offload_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config_name: str):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary, if it
+    was captured on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(config_name)
+    if not e or e.get("src_hash") != src_hash("dkv_attention.cu", "dkv_common.cuh"):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU workload
+
+
+def gpu_randn_bf16(shape, gen, std=1.0, device="cuda"):
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    flat = out.view(-1)
+    n = flat.numel()
+    step = 1 << 26
+    for s in range(0, n, step):
+        e = min(n, s + step)
+        v = torch.randn(e - s, generator=gen, device=device, dtype=torch.float32)
+        if std != 1.0:
+            v.mul_(std)
+        flat[s:e].copy_(v)
+    return out
+
+
+class Workload:
+    """A decode workload resident on one GPU: pool (both tiers filled), tables, x, W."""
+
+    def __init__(self, cfg: WL.DecodeConfig, seed: int, host_flags: int = 0):
+        import kv_cache_offload_b200 as dkv
+        self.dkv = dkv
+        self.cfg = cfg
+        dev = torch.device("cuda", torch.cuda.current_device())
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed)
+        self.lay = WL.block_layout(cfg, seed)
+        lay = self.lay
+        tier_elems = cfg.layers * 2 * cfg.Hkv * cfg.T * cfg.D
+        self.hbm = gpu_randn_bf16((lay.hbm_blocks * tier_elems,), gen) if lay.hbm_blocks else None
+        self.pool = dkv.dkv_pool_create(cfg.layers, cfg.Hkv, cfg.D, lay.hbm_blocks, lay.host_blocks,
+                                        host_flags=host_flags, hbm_base=self.hbm)
+        if lay.host_blocks:
+            host = dkv.host_tier_tensor(self.pool)
+            n = host.numel()
+            step = 1 << 28
+            for s in range(0, n, step):
+                e = min(n, s + step)
+                host[s:e].copy_(gpu_randn_bf16((e - s,), gen).view(torch.int16).cpu())
+        self.x = gpu_randn_bf16((cfg.B, cfg.H), gen)
+        self.W = gpu_randn_bf16((cfg.rows, cfg.H), gen, std=1.0 / math.sqrt(cfg.H))
+        self.table = lay.block_table.to(dev)
+        self.tmap = lay.tier_map.to(dev)
+        self.lens = torch.tensor(lay.seq_lens, dtype=torch.int32, device=dev)
+        self.out = torch.empty((cfg.B, cfg.Hq * cfg.D), dtype=torch.bfloat16, device=dev)
+        self.nws = dkv.dkv_decode_workspace_bytes(self.pool, cfg.B, lay.max_blocks, cfg.Hq, cfg.H)
+        self.ws = torch.empty(self.nws, dtype=torch.uint8, device=dev)
+        # byte accounting (algorithmic: what the step must move)
+        per_tok = 2 * cfg.Hkv * cfg.D * 2          # K and V of one token, all kv heads
+        host_tok = hbm_tok = 0
+        for b, c in enumerate(lay.seq_lens):
+            for j in range((c + cfg.T - 1) // cfg.T):
+                n = min(cfg.T, c - j * cfg.T)
+                if int(lay.tier_map[b, j]):
+                    host_tok += n
+                else:
+                    hbm_tok += n
+        self.kv_host_bytes = host_tok * per_tok
+        self.kv_hbm_bytes = hbm_tok * per_tok
+        self.kv_bytes = self.kv_host_bytes + self.kv_hbm_bytes
+        self.w_bytes = cfg.rows * cfg.H * 2
+        self.new_kv_bytes = cfg.B * cfg.Hkv * cfg.D * 2 * 2
+        self.splits = dkv.dkv_decode_attn_splits(self.pool, cfg.B, lay.max_blocks, cfg.Hq)
+
+    def set_tuning(self, attn_splits=0, proj_splits=0):
+        self.dkv.dkv_pool_set_tuning(self.pool, attn_splits=attn_splits, proj_splits=proj_splits)
+        self.splits = self.dkv.dkv_decode_attn_splits(self.pool, self.cfg.B, self.lay.max_blocks,
+                                                      self.cfg.Hq)
+
+    def step(self):
+        c = self.cfg
+        self.dkv.dkv_decode_step(self.pool, 0, self.x, self.W, self.table, self.lens, self.tmap, c.Hq,
+                                 c.theta, self.out, self.ws)
+
+    def step_timed_stages(self, ev):
+        c, d = self.cfg, self.dkv
+        ev[0].record()
+        d.dkv_decode_project(self.pool, 0, self.x, self.W, self.table, self.lens, self.tmap, c.Hq,
+                             c.theta, self.ws)
+        ev[1].record()
+        d.dkv_decode_attend(self.pool, 0, self.table, self.lens, self.tmap, c.H, c.Hq, self.ws)
+        ev[2].record()
+        d.dkv_decode_combine(self.pool, c.B, self.lay.max_blocks, c.H, c.Hq, self.out, self.ws)
+        ev[3].record()
+
+    def close(self):
+        if self.pool:
+            self.dkv.dkv_pool_destroy(self.pool)
+            self.pool = 0
+
+
+def measure_h2d_peak(dev, nbytes=1 << 30, reps=5):
+    src = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    dst.copy_(src, non_blocking=True)
+    torch.cuda.synchronize()
+    best = 0.0
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        dst.copy_(src, non_blocking=True)
+        b.record()
+        b.synchronize()
+        best = max(best, nbytes / (a.elapsed_time(b) * 1e-3) / 1e9)
+    del src, dst
+    return best
+
+
+# -------------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(cfg: WL.DecodeConfig, seed: int, n_seq: int):
+    """A bounded sample of the workload for the oracle: the first n_seq sequences' shapes
+    (same lengths, tiers, block counts), generated on the host."""
+    sub = WL.DecodeConfig(cfg.name, B=n_seq, H=cfg.H, Hq=cfg.Hq, Hkv=cfg.Hkv, D=cfg.D,
+                          theta=cfg.theta, ctx=cfg.ctx, ctx_range=cfg.ctx_range,
+                          tier_policy=cfg.tier_policy, recent_hbm_tokens=cfg.recent_hbm_tokens,
+                          host_prob=cfg.host_prob, permute=cfg.permute, layers=cfg.layers, T=cfg.T)
+    lens = WL.seq_lengths(cfg, seed)[:n_seq]
+    return WL.make_decode_inputs(sub, seed=seed, seq_lens=lens)
+
+
+def time_oracle(inp, budget_s: float):
+    """Run the oracle sequence by sequence until the budget is spent; tokens/s."""
+    from oracle import dkv_oracle as O
+    cfg, lay = inp.cfg, inp.layout
+    xb, Wb = WL.bf16_bits(inp.x), WL.bf16_bits(inp.W)
+    tiers = [WL.bf16_bits(inp.hbm), WL.bf16_bits(inp.host)]
+    done, t0 = 0, time.perf_counter()
+    for b in range(cfg.B):
+        O.decode_step(xb, Wb, tiers, lay.block_table.numpy(), lay.seq_lens, lay.tier_map.numpy(),
+                      cfg.Hq, cfg.Hkv, cfg.D, cfg.T, cfg.theta, batch=[b])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    el = time.perf_counter() - t0
+    return done / el, done, el
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return 1
+
+
+def cpu_baseline(cfg, seed, budget_s):
+    n_seq = max(1, min(cfg.B, 4))
+    inp = oracle_sample(cfg, seed, n_seq)
+    rate, done, el = time_oracle(inp, budget_s)
+    return {"value": rate, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+            "sample": "%d of %d sequences of the same workload (full context each), %.1f s of fp64 "
+                      "numpy oracle work" % (done, cfg.B, el)}
+
+
+# --------------------------------------------------------------------------- main
+
+
+def run_reference(args, rank, world):
+    cfg = WL.CONFIGS[args.config]
+    if rank != 0:
+        return
+    inp = oracle_sample(cfg, 0, 1)
+    times = []
+    for i in range(args.warmup + args.steps):
+        rate, done, el = time_oracle(inp, 0.0)
+        if i >= args.warmup:
+            times.append(el)
+    ms = 1e3 * sum(times) / len(times)
+    value = 1.0 / (ms * 1e-3)
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": cfg.name, "B": cfg.B, "hidden": cfg.H, "Hq": cfg.Hq, "Hkv": cfg.Hkv,
+                       "head_dim": cfg.D, "step_sample": "1 sequence of the workload per step"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
+                             "sample": "1 of %d sequences per step (full context)" % cfg.B},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = world > 1
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.warmup < 3:
+        args.warmup = 3
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if dist:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=dev)
+    from kv_cache_offload_b200.build import build
+    if rank == 0 or not dist:
+        build()
+    if dist:
+        tdist.barrier()
+    import kv_cache_offload_b200 as dkv
+
+    cfg = WL.CONFIGS[args.config]
+    wl = Workload(cfg, seed=rank, host_flags=args.host_flags)
+    wl.set_tuning(args.attn_splits, args.proj_splits)
+
+    def barrier():
+        if dist:
+            tdist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        wl.step()
+    assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
+
+    # ---- value: K back-to-back steps, inputs resident in HBM / host tier
+    clocks = ClockSampler(local)
+    barrier()
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        wl.step()
+    e1.record()
+    barrier()
+    clk = clocks.stop()
+    t_ms = e0.elapsed_time(e1)
+    assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
+
+    # ---- per-stage durations (same steps with events between the three launches)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        wl.step_timed_stages(evs[i])
+    barrier()
+    stage_ms = [sum(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)) / args.steps
+                for k in range(3)]
+
+    # ---- e2e: host buffers in, result out, through the public API
+    xh = wl.x.cpu().pin_memory()
+    th, mh, lh = wl.table.cpu().pin_memory(), wl.tmap.cpu().pin_memory(), wl.lens.cpu().pin_memory()
+    oh = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+    xd, td, md, ld = torch.empty_like(wl.x), torch.empty_like(wl.table), torch.empty_like(wl.tmap), \
+        torch.empty_like(wl.lens)
+    h2d = xh.numel() * 2 + th.numel() * 4 + mh.numel() + lh.numel() * 4
+    d2h = oh.numel() * 2
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        xd.copy_(xh, non_blocking=True); td.copy_(th, non_blocking=True)
+        md.copy_(mh, non_blocking=True); ld.copy_(lh, non_blocking=True)
+        dkv.dkv_decode_step(wl.pool, 0, xd, wl.W, td, ld, md, cfg.Hq, cfg.theta, wl.out, wl.ws)
+        oh.copy_(wl.out, non_blocking=True)
+    b.record()
+    barrier()
+    e2e_ms = a.elapsed_time(b)
+
+    # ---- max over ranks
+    vals = torch.tensor([t_ms, e2e_ms] + stage_ms, dtype=torch.float64, device=dev)
+    if dist:
+        tdist.all_reduce(vals, op=tdist.ReduceOp.MAX)
+    t_ms, e2e_ms = float(vals[0]), float(vals[1])
+    stage_ms = [float(v) for v in vals[2:]]
+    ms = t_ms / args.steps
+    tokens = cfg.B * world
+    value = tokens / (ms * 1e-3)
+    e2e_val = tokens / (e2e_ms / args.steps * 1e-3)
+
+    peak, peak_kind = load_peaks()
+    attn_ms = stage_ms[1]
+    achieved = wl.kv_bytes / (attn_ms * 1e-3) / 1e9
+    host_info = None
+    if wl.kv_host_bytes:
+        h2d_peak = measure_h2d_peak(dev)
+        host_gbs = wl.kv_host_bytes / (attn_ms * 1e-3) / 1e9
+        host_info = {"h2d_peak_gbs": h2d_peak, "host_kv_bytes": wl.kv_host_bytes,
+                     "achieved_gbs": host_gbs, "frac": host_gbs / h2d_peak,
+                     "link": "PCIe (not NVLink-C2C)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "%s: B=%d hidden=%d Hq=%d Hkv=%d D=%d theta=%g, cached tokens %s, "
+                               "%d-token blocks, tiers %s" % (cfg.name, cfg.B, cfg.H, cfg.Hq, cfg.Hkv, cfg.D,
+                                                              cfg.theta, cfg.ctx or cfg.ctx_range, cfg.T,
+                                                              cfg.tier_policy),
+                   "global_batch": cfg.B * world, "seq_len": cfg.ctx or max(wl.lay.seq_lens),
+                   "parallelism": "replicas x%d" % world, "attn_splits": wl.splits,
+                   "l2": "inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)},
+        "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
+        "stage_ms": {"project": stage_ms[0], "attend": stage_ms[1], "combine": stage_ms[2]},
+        "roofline": {"bound": "hbm" if not wl.kv_host_bytes else "host_link", "kernel": "attn_splitk_kernel",
+                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_source": peak_kind,
+                     "traffic": profiled_traffic(cfg.name),
+                     "algorithmic_bytes_per_launch": wl.kv_bytes},
+        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clk,
+    }
+    if host_info:
+        line["host_link"] = host_info
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, 0, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    wl.close()
+    if dist:
+        tdist.barrier()
+        tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+/*
+ * dkv.h — C ABI of libdkv: a zero-copy, two-tier paged KV cache and the fused decode step
+ * (QKV projection + RoPE + GQA split-K decode attention) for NVIDIA B200 (sm_100a).
+ *
+ * The problem these calls follow is DirectKV's ("长上下文 LLM 的零拷贝 KV Cache 卸载（OSDI
+ * 2026）", sections 问题与动机 and 核心方法): conventional KV offload stages host-resident KV
+ * blocks into an HBM buffer before attention reads them, which costs GPU capacity and
+ * moves the data twice; DirectKV lets the attention kernel read CPU-resident KV in place,
+ * fuses the QKV projection with attention so the new K/V are consumed on chip and written
+ * once, and overlaps fetch with compute in a warp-level pipeline. The paged-block pool and
+ * the block table are the usual PagedAttention structures ("KV Offload" wiki page,
+ * sections Swap-out / Swap-in: blocks are the unit that is freed and moved).
+ *
+ * Conventions shared by every call:
+ *  - bf16 tensors are passed as `uint16_t*` holding raw bf16 bit patterns.
+ *  - "device pointer" means an address the current CUDA device can dereference: device
+ *    memory, or the device alias of mapped pinned host memory.
+ *  - `stream` is a `cudaStream_t` passed as `void*` (NULL = the legacy default stream).
+ *    Every call that takes a stream only enqueues work on it and never synchronises,
+ *    except dkv_check and the pool create/destroy calls.
+ *  - Return value: DKV_OK (0) or a negative DKV_ERR_* code. Nothing throws across the ABI.
+ *    dkv_last_error() returns a thread-local message for the last failing call.
+ *  - The library owns the pool and both tiers (unless `hbm_base` is supplied); the
+ *    caller owns every other buffer (inputs, tables, outputs, workspaces).
+ *  - Device-detected faults (bad tier value, physical block id out of range, a context
+ *    longer than the block table) never trap: the kernel skips the offending block, sets
+ *    a bit in the pool's status word, and dkv_check() reports DKV_ERR_BAD_TABLE.
+ */
+#ifndef DKV_H_
+#define DKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DKV_OK               0
+#define DKV_ERR_ARG         (-1)  /* invalid argument (null pointer, bad size, bad enum) */
+#define DKV_ERR_CUDA        (-2)  /* a CUDA runtime/driver call failed */
+#define DKV_ERR_OOM         (-3)  /* device or pinned-host allocation failed */
+#define DKV_ERR_UNSUPPORTED (-4)  /* shape/device not supported (see each call) */
+#define DKV_ERR_BAD_TABLE   (-5)  /* device-side table validation failed (dkv_check) */
+#define DKV_ERR_TIMEOUT     (-6)  /* a bounded device-side wait gave up (dkv_check) */
+#define DKV_ERR_CAPACITY    (-7)  /* request exceeds a fixed capacity */
+
+#define DKV_TIER_HBM  0
+#define DKV_TIER_HOST 1
+
+#define DKV_LAYOUT_LAYER_FIRST 0  /* tier = [L][P][2][Hkv][T][D] */
+#define DKV_LAYOUT_PAGE_FIRST  1  /* tier = [P][L][2][Hkv][T][D] */
+
+#define DKV_HOST_WRITE_COMBINED 1 /* host tier allocated write-combined */
+
+typedef struct dkv_pool dkv_pool;  /* opaque; owned by the library */
+
+/*
+ * Pool geometry. One physical block holds T consecutive tokens of one sequence for every
+ * layer, both K and V, every kv head: per (layer, block, K|V, kv head) a contiguous
+ * [T][D] bf16 chunk (4 KiB at T=16, D=128). DirectKV reorders the KV layout so that reads
+ * of CPU-resident KV coalesce (核心方法); contiguous per-head chunks are that layout here.
+ * The two layouts are Strata's layer-first / page-first decoupling ("「KV Cache 内存层级」
+ * 系列总纲", §2.4 Strata).
+ */
+typedef struct dkv_pool_config {
+  int32_t num_layers;    /* L >= 1 */
+  int32_t num_kv_heads;  /* Hkv >= 1 */
+  int32_t head_dim;      /* D: 64 or 128 */
+  int32_t block_tokens;  /* T: 16 */
+  int64_t hbm_blocks;    /* physical blocks in the HBM tier (>= 0) */
+  int64_t host_blocks;   /* physical blocks in the host tier (>= 0) */
+  int32_t layout;        /* DKV_LAYOUT_* */
+  int32_t host_flags;    /* 0 or DKV_HOST_WRITE_COMBINED */
+  void*   hbm_base;      /* optional caller-owned device buffer of at least the HBM tier's
+                            size (256-byte aligned); NULL = the library allocates it */
+} dkv_pool_config;
+
+/* Launch tunables; 0 means "choose automatically". */
+typedef struct dkv_tuning {
+  int32_t attn_splits;   /* split-K factor of the attention grid (per sequence, kv head) */
+  int32_t proj_splits;   /* split factor of the projection's reduction dimension */
+  int32_t reserved[6];
+} dkv_tuning;
+
+/*
+ * Create a pool on the current device: the HBM tier (device memory) and the host tier
+ * (pinned host memory allocated mapped, so kernels read it in place through its device
+ * alias with no staging copy: DirectKV 核心方法). Requires an sm_100 device.
+ * Errors: DKV_ERR_ARG (bad geometry), DKV_ERR_UNSUPPORTED (D not 64/128, T != 16, not
+ * sm_100), DKV_ERR_OOM (either allocation failed; nothing is leaked).
+ * Tier contents are uninitialised.
+ */
+int dkv_pool_create(const dkv_pool_config* cfg, dkv_pool** out);
+
+/* Free both tiers (not a caller-supplied hbm_base) and the pool. Synchronises the device. */
+int dkv_pool_destroy(dkv_pool* pool);
+
+/*
+ * Base address and size in bytes of a tier. For DKV_TIER_HOST, `*dev_ptr` is the device
+ * alias; `host_ptr` (may be NULL) receives the host-side address of the same memory.
+ */
+int dkv_pool_tier_ptr(const dkv_pool* pool, int tier, void** dev_ptr, void** host_ptr,
+                      size_t* bytes);
+
+/* Set launch tunables for later calls on this pool (copied). NULL restores defaults. */
+int dkv_pool_set_tuning(dkv_pool* pool, const dkv_tuning* tuning);
+
+/*
+ * Append n_tokens new tokens per sequence (e.g. a prefill's K/V) into the cache.
+ * k, v: device [B][n_tokens][Hkv][D] bf16. Token t of sequence b goes to position
+ * seq_lens[b] + t: slot (pos mod T) of logical block floor(pos / T), which lives in tier
+ * tier_map[b*max_blocks + j] at physical index block_table[b*max_blocks + j].
+ * block_table (int32), seq_lens (int32), tier_map (uint8) are device arrays. seq_lens is
+ * not modified. Bad table entries are skipped and flagged (see dkv_check).
+ */
+int dkv_append_kv(dkv_pool* pool, int layer, const uint16_t* k, const uint16_t* v, int B,
+                  int n_tokens, const int32_t* block_table, int max_blocks,
+                  const int32_t* seq_lens, const uint8_t* tier_map, void* stream);
+
+/* Bytes of caller-provided workspace dkv_decode_step needs for this shape. */
+size_t dkv_decode_workspace_bytes(const dkv_pool* pool, int B, int max_blocks,
+                                  int num_q_heads, int hidden);
+
+/*
+ * One decode step of one layer for a batch of B sequences (DirectKV 核心方法: QKV
+ * projection fused with attention over CPU-resident KV, no staging buffer):
+ *   qkv_b = Wqkv . x_b (no norm, no bias); rows [Hq q heads][Hkv k heads][Hkv v heads] x D
+ *   q, k rotated by RoPE (rotate-half pairs (i, i+D/2), angle pos * theta^(-2i/D)) at
+ *   pos = seq_lens[b];
+ *   k_hat = bf16(k_rot), v_hat = bf16(v) written once into slot pos mod T of logical
+ *   block floor(pos/T) (the table must cover ceil((pos+1)/T) blocks);
+ *   out_b[h] = softmax over keys 0..pos of (q_h . k_t / sqrt(D)) applied to v_t, with
+ *   q head h attending kv head h / (Hq/Hkv); keys 0..pos-1 come from the cache (either
+ *   tier, read in place), key pos is (k_hat, v_hat).
+ * x: device [B][hidden] bf16. Wqkv: device [(Hq+2Hkv)*D][hidden] bf16, row-major.
+ * block_table: device int32 [B][max_blocks]; tier_map: device uint8 [B][max_blocks]
+ * (0 = HBM, 1 = host); seq_lens: device int32 [B] (cached tokens; NOT incremented).
+ * out: device [B][Hq*D] bf16. workspace: device, >= dkv_decode_workspace_bytes(...),
+ * 256-byte aligned; its contents need no initialisation.
+ * Supported: 1 <= B <= 32, hidden % 64 == 0, Hq % Hkv == 0 with Hq/Hkv in {1,2,4,8}.
+ * Three stream-ordered kernels (projection, attention, combine); no host synchronisation,
+ * no allocation, so the call can be captured into a CUDA graph.
+ */
+int dkv_decode_step(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t* Wqkv,
+                    const int32_t* block_table, const int32_t* seq_lens,
+                    const uint8_t* tier_map, int B, int max_blocks, int hidden,
+                    int num_q_heads, float rope_theta, uint16_t* out, void* workspace,
+                    size_t ws_bytes, void* stream);
+
+/*
+ * The three stages of dkv_decode_step as separate calls, with the same arguments and the
+ * same workspace (for timing each stage). dkv_decode_step == project; attend; combine.
+ *   project: projection, RoPE, the single cache write, the new token's partial softmax
+ *            state (score and value), q for the attention — all into the workspace.
+ *   attend:  split-K partial softmax states over the cached blocks of both tiers.
+ *   combine: merges the partial states and the new token's into out (bf16).
+ */
+int dkv_decode_project(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t* Wqkv,
+                       const int32_t* block_table, const int32_t* seq_lens,
+                       const uint8_t* tier_map, int B, int max_blocks, int hidden,
+                       int num_q_heads, float rope_theta, void* workspace, size_t ws_bytes,
+                       void* stream);
+int dkv_decode_attend(dkv_pool* pool, int layer, const int32_t* block_table,
+                      const int32_t* seq_lens, const uint8_t* tier_map, int B,
+                      int max_blocks, int hidden, int num_q_heads, void* workspace,
+                      size_t ws_bytes, void* stream);
+int dkv_decode_combine(dkv_pool* pool, int B, int max_blocks, int hidden, int num_q_heads,
+                       uint16_t* out, void* workspace, size_t ws_bytes, void* stream);
+
+/* The attention split-K factor dkv_decode_step uses for this shape (after tuning). */
+int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
+
+/*
+ * Block-layout permutation (Strata's layout decoupling with GPU-driven copy: "「KV Cache
+ * 内存层级」系列总纲", §2.4 Strata): copy `src` laid out as [A][Bn][chunk] into `dst` as
+ * [Bn][A][chunk], where for src_layout == DKV_LAYOUT_LAYER_FIRST A = num_layers and
+ * Bn = num_blocks (result page-first), and for DKV_LAYOUT_PAGE_FIRST A = num_blocks and
+ * Bn = num_layers (result layer-first). chunk_bytes = 2 * Hkv * T * D * 2 (one block of
+ * one layer), a multiple of 16. src and dst are device pointers (either may be the device
+ * alias of mapped host memory), 16-byte aligned, not overlapping. Bit-exact.
+ */
+int dkv_permute_layout(const void* src, void* dst, int src_layout, int num_layers,
+                       int64_t num_blocks, int64_t chunk_bytes, void* stream);
+
+/* Convert a whole tier of the pool into the other layout, written to `dst`
+ * (dst_bytes >= the tier's size). The pool itself is not modified. */
+int dkv_convert_layout(dkv_pool* pool, int tier, void* dst, size_t dst_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the pool's device status word.
+ * Returns DKV_OK, DKV_ERR_BAD_TABLE (a kernel skipped a block with a bad tier or physical
+ * id, or a context exceeding max_blocks*T), DKV_ERR_TIMEOUT, or DKV_ERR_CUDA.
+ */
+int dkv_check(dkv_pool* pool, void* stream);
+
+/* Thread-local message describing the last failing call on this thread ("" if none). */
+const char* dkv_last_error(void);
+
+/* Library version string. */
+const char* dkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DKV_H_ */

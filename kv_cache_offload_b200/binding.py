@@ -1,0 +1,274 @@
+"""ctypes binding of libdkv's C ABI (include/dkv.h), one Python function per C entry point
+with the same name. Argument marshalling only: tensors are passed as raw pointers, the
+current torch CUDA stream as the stream handle, and every computation happens in the
+library's kernels. If the library is missing the calls raise; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdkv.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "dkv.h")
+
+DKV_OK = 0
+DKV_ERR_ARG = -1
+DKV_ERR_CUDA = -2
+DKV_ERR_OOM = -3
+DKV_ERR_UNSUPPORTED = -4
+DKV_ERR_BAD_TABLE = -5
+DKV_ERR_TIMEOUT = -6
+DKV_ERR_CAPACITY = -7
+
+DKV_TIER_HBM = 0
+DKV_TIER_HOST = 1
+DKV_LAYOUT_LAYER_FIRST = 0
+DKV_LAYOUT_PAGE_FIRST = 1
+DKV_HOST_WRITE_COMBINED = 1
+
+
+class DkvError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("dkv error %d: %s" % (code, msg))
+        self.code = code
+
+
+class dkv_pool_config(ctypes.Structure):
+    _fields_ = [("num_layers", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("block_tokens", ctypes.c_int32),
+                ("hbm_blocks", ctypes.c_int64), ("host_blocks", ctypes.c_int64),
+                ("layout", ctypes.c_int32), ("host_flags", ctypes.c_int32),
+                ("hbm_base", ctypes.c_void_p)]
+
+
+class dkv_tuning(ctypes.Structure):
+    _fields_ = [("attn_splits", ctypes.c_int32), ("proj_splits", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 6)]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_F = ctypes.c_float
+
+_SIGS = {
+    "dkv_pool_create": (_I, [ctypes.POINTER(dkv_pool_config), ctypes.POINTER(_P)]),
+    "dkv_pool_destroy": (_I, [_P]),
+    "dkv_pool_tier_ptr": (_I, [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_SZ)]),
+    "dkv_pool_set_tuning": (_I, [_P, ctypes.POINTER(dkv_tuning)]),
+    "dkv_append_kv": (_I, [_P, _I, _P, _P, _I, _I, _P, _I, _P, _P, _P]),
+    "dkv_decode_workspace_bytes": (_SZ, [_P, _I, _I, _I, _I]),
+    "dkv_decode_step": (_I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _SZ, _P]),
+    "dkv_decode_project": (_I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _SZ, _P]),
+    "dkv_decode_attend": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "dkv_decode_combine": (_I, [_P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
+    "dkv_decode_attn_splits": (_I, [_P, _I, _I, _I]),
+    "dkv_permute_layout": (_I, [_P, _P, _I, _I, _I64, _I64, _P]),
+    "dkv_convert_layout": (_I, [_P, _I, _P, _SZ, _P]),
+    "dkv_check": (_I, [_P, _P]),
+    "dkv_last_error": (ctypes.c_char_p, []),
+    "dkv_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdkv.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libdkv.so is not built (%s); run kv_cache_offload_b200.build.build()" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def header_symbols(path: str = HEADER):
+    """Names of the functions include/dkv.h declares."""
+    txt = open(path).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(dkv_[a-z_0-9]+)\s*\(", txt)))
+
+
+def dkv_last_error() -> str:
+    return lib().dkv_last_error().decode()
+
+
+def dkv_version() -> str:
+    return lib().dkv_version().decode()
+
+
+def _chk(rc: int):
+    if rc != DKV_OK:
+        raise DkvError(rc, dkv_last_error())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        if torch.cuda.is_available():
+            return torch.cuda.current_stream().cuda_stream
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _need(t: torch.Tensor, dtype, name: str, cuda: bool = True):
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s (got %s)" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if cuda and not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+
+
+# ------------------------------------------------------------------------- pool
+
+
+def dkv_pool_create(num_layers: int, num_kv_heads: int, head_dim: int, hbm_blocks: int,
+                    host_blocks: int, block_tokens: int = 16, layout: int = 0,
+                    host_flags: int = 0, hbm_base: Optional[torch.Tensor] = None) -> int:
+    cfg = dkv_pool_config(num_layers, num_kv_heads, head_dim, block_tokens, hbm_blocks,
+                          host_blocks, layout, host_flags, _ptr(hbm_base))
+    out = _P()
+    _chk(lib().dkv_pool_create(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def dkv_pool_destroy(pool: int):
+    _chk(lib().dkv_pool_destroy(pool))
+
+
+def dkv_pool_tier_ptr(pool: int, tier: int):
+    """(device pointer, host pointer or None, bytes) of a tier."""
+    d, h, n = _P(), _P(), _SZ()
+    _chk(lib().dkv_pool_tier_ptr(pool, tier, ctypes.byref(d), ctypes.byref(h), ctypes.byref(n)))
+    return d.value, h.value, n.value
+
+
+def dkv_pool_set_tuning(pool: int, attn_splits: int = 0, proj_splits: int = 0):
+    t = dkv_tuning(attn_splits, proj_splits)
+    _chk(lib().dkv_pool_set_tuning(pool, ctypes.byref(t)))
+
+
+def host_tier_tensor(pool: int) -> torch.Tensor:
+    """The host tier as a flat CPU int16 tensor (raw bf16 bits) aliasing the pinned memory."""
+    _, h, n = dkv_pool_tier_ptr(pool, DKV_TIER_HOST)
+    if not n:
+        return torch.empty(0, dtype=torch.int16)
+    buf = (ctypes.c_int16 * (n // 2)).from_address(h)
+    import numpy as np
+    return torch.from_numpy(np.ctypeslib.as_array(buf))
+
+
+def dkv_append_kv(pool: int, layer: int, k: torch.Tensor, v: torch.Tensor,
+                  block_table: torch.Tensor, seq_lens: torch.Tensor, tier_map: torch.Tensor,
+                  stream=None):
+    """k, v: [B, n_tokens, Hkv, D] bf16 on the device."""
+    _need(k, torch.bfloat16, "k"); _need(v, torch.bfloat16, "v")
+    _need(block_table, torch.int32, "block_table"); _need(seq_lens, torch.int32, "seq_lens")
+    _need(tier_map, torch.uint8, "tier_map")
+    B, n = k.shape[0], k.shape[1]
+    _chk(lib().dkv_append_kv(pool, layer, _ptr(k), _ptr(v), B, n, _ptr(block_table),
+                             block_table.shape[1], _ptr(seq_lens), _ptr(tier_map), _stream(stream)))
+
+
+# ---------------------------------------------------------------------- decode
+
+
+def dkv_decode_workspace_bytes(pool: int, B: int, max_blocks: int, num_q_heads: int, hidden: int) -> int:
+    n = lib().dkv_decode_workspace_bytes(pool, B, max_blocks, num_q_heads, hidden)
+    if n == 0:
+        raise DkvError(DKV_ERR_ARG, dkv_last_error())
+    return n
+
+
+def dkv_decode_attn_splits(pool: int, B: int, max_blocks: int, num_q_heads: int) -> int:
+    r = lib().dkv_decode_attn_splits(pool, B, max_blocks, num_q_heads)
+    if r < 0:
+        raise DkvError(r, dkv_last_error())
+    return r
+
+
+def _decode_checks(x, Wqkv, block_table, seq_lens, tier_map):
+    _need(x, torch.bfloat16, "x"); _need(Wqkv, torch.bfloat16, "Wqkv")
+    _need(block_table, torch.int32, "block_table"); _need(seq_lens, torch.int32, "seq_lens")
+    _need(tier_map, torch.uint8, "tier_map")
+    if block_table.shape != tier_map.shape or block_table.shape[0] != x.shape[0]:
+        raise ValueError("block_table/tier_map must be [B, max_blocks] with B = x.shape[0]")
+
+
+def dkv_decode_step(pool: int, layer: int, x: torch.Tensor, Wqkv: torch.Tensor,
+                    block_table: torch.Tensor, seq_lens: torch.Tensor, tier_map: torch.Tensor,
+                    num_q_heads: int, rope_theta: float, out: torch.Tensor,
+                    workspace: torch.Tensor, stream=None):
+    _decode_checks(x, Wqkv, block_table, seq_lens, tier_map)
+    _need(out, torch.bfloat16, "out")
+    B, H = x.shape
+    _chk(lib().dkv_decode_step(pool, layer, _ptr(x), _ptr(Wqkv), _ptr(block_table), _ptr(seq_lens),
+                               _ptr(tier_map), B, block_table.shape[1], H, num_q_heads,
+                               float(rope_theta), _ptr(out), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dkv_decode_project(pool, layer, x, Wqkv, block_table, seq_lens, tier_map, num_q_heads,
+                       rope_theta, workspace, stream=None):
+    _decode_checks(x, Wqkv, block_table, seq_lens, tier_map)
+    B, H = x.shape
+    _chk(lib().dkv_decode_project(pool, layer, _ptr(x), _ptr(Wqkv), _ptr(block_table), _ptr(seq_lens),
+                                  _ptr(tier_map), B, block_table.shape[1], H, num_q_heads,
+                                  float(rope_theta), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dkv_decode_attend(pool, layer, block_table, seq_lens, tier_map, hidden, num_q_heads,
+                      workspace, stream=None):
+    B = block_table.shape[0]
+    _chk(lib().dkv_decode_attend(pool, layer, _ptr(block_table), _ptr(seq_lens), _ptr(tier_map), B,
+                                 block_table.shape[1], hidden, num_q_heads, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dkv_decode_combine(pool, B, max_blocks, hidden, num_q_heads, out, workspace, stream=None):
+    _need(out, torch.bfloat16, "out")
+    _chk(lib().dkv_decode_combine(pool, B, max_blocks, hidden, num_q_heads, _ptr(out), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+# ---------------------------------------------------------------------- layout
+
+
+def dkv_permute_layout(src, dst, src_layout: int, num_layers: int, num_blocks: int,
+                       chunk_bytes: int, stream=None):
+    _chk(lib().dkv_permute_layout(_ptr(src), _ptr(dst), src_layout, num_layers, num_blocks,
+                                  chunk_bytes, _stream(stream)))
+
+
+def dkv_convert_layout(pool: int, tier: int, dst, dst_bytes: Optional[int] = None, stream=None):
+    if dst_bytes is None:
+        dst_bytes = dst.numel() * dst.element_size()
+    _chk(lib().dkv_convert_layout(pool, tier, _ptr(dst), dst_bytes, _stream(stream)))
+
+
+def dkv_check(pool: int, stream=None) -> int:
+    """Synchronise and return the pool's status code (DKV_OK or a DKV_ERR_*)."""
+    return lib().dkv_check(pool, _stream(stream))

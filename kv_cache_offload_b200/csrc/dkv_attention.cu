@@ -1,0 +1,414 @@
+// Split-K GQA decode attention over a two-tier paged KV cache, and the split combine.
+//
+// DirectKV ("长上下文 LLM 的零拷贝 KV Cache 卸载（OSDI 2026）", 核心方法) lets the attention
+// kernel read CPU-resident KV in place and hides the slow fetches behind compute with a
+// warp-level producer/consumer pipeline. This kernel is that pipeline on sm_100a:
+//
+//  * one CTA per (split s, kv head g, sequence b) walks a contiguous range of logical
+//    blocks; the KV of kv head g is read once for all G = Hq/Hkv query heads;
+//  * one producer warp fills an NST-stage shared-memory ring, one stage per block
+//    (K chunk [T][D] then V chunk [T][D], both contiguous in the pool):
+//      - HBM-tier block: one lane issues two bulk copies (TMA engine) of the chunks;
+//      - host-tier block: all 32 lanes issue 16-byte cp.async loads straight from the
+//        mapped pinned host memory (coalesced 512-byte warp requests), no staging buffer;
+//    both complete on the stage's mbarrier, so the consumers see one kind of stage;
+//  * four consumer "slots" (WPB warps each; heads split across the WPB warps) take
+//    blocks round robin, each keeping its own online-softmax state (running max m,
+//    running sum l, accumulator acc) in registers; the slots merge at the end and the CTA
+//    writes one partial state (m, l, acc[D]) per q head to the workspace.
+//
+// Scores are computed in the log2 domain: q arrives pre-scaled by log2(e)/sqrt(D), so
+// p = 2^(s - m). Arithmetic is fp32 on CUDA cores (a decode query is a handful of rows:
+// G flops per byte of KV, HBM-bound, not a tensor-core contraction).
+#include <math.h>
+
+#include "dkv_internal.h"
+
+namespace dkv {
+
+constexpr int kSlots = 4;
+constexpr int kT = 16;
+
+template <int D, int HPW, int WPB, int NST>
+struct AttnCfg {
+  static constexpr int G = HPW * WPB;
+  static constexpr int NCW = kSlots * WPB;  // consumer warps
+  static constexpr int THREADS = (NCW + 1) * 32;
+  static constexpr int STAGE_ELEMS = 2 * kT * D;
+  static constexpr int STAGE_BYTES = STAGE_ELEMS * 2;
+  static constexpr int DPL = D / 32;   // value dims per lane in P.V
+  static constexpr int QCH = D / 64;   // 16-byte key chunks per lane per token in Q.K
+  static constexpr int NV = HPW * 4;   // partial scores per lane (heads x 4 tokens)
+  static constexpr int LOGH = HPW == 4 ? 2 : (HPW == 2 ? 1 : 0);
+  static constexpr int LOWMASK = (1 << (3 - LOGH)) - 1;  // dg bits shared by one head
+  static constexpr int NR = NV >= 8 ? NV / 8 : 1;        // scores per lane after reduction
+  static constexpr int OFF_P = NST * STAGE_BYTES;
+  static constexpr int OFF_ALPHA = OFF_P + NCW * kT * HPW * 4;
+  static constexpr int OFF_FLAGS = OFF_ALPHA + NCW * HPW * 4;
+  static constexpr int OFF_BARS = (OFF_FLAGS + NST * 4 + 7) / 8 * 8;
+  static constexpr int SMEM = OFF_BARS + 2 * NST * 8;
+  static constexpr int MERGE_BYTES = NCW * HPW * D * 4 + NCW * HPW * 8;
+  static_assert(MERGE_BYTES <= NST * STAGE_BYTES, "merge area must fit in the stage ring");
+  static_assert(NST >= kSlots, "ring must hold one block per consumer slot");
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// One level of a warp reduce-scatter: lanes with `up` keep the upper half of the N live
+// values, their partner (lane ^ mask) the lower half; each adds the partner's copy.
+template <int N>
+__device__ __forceinline__ void rs_level(float* v, bool up, int mask) {
+  if constexpr (N >= 2) {
+#pragma unroll
+    for (int x = 0; x < N / 2; ++x) {
+      const float send = up ? v[x] : v[x + N / 2];
+      const float keep = up ? v[x + N / 2] : v[x];
+      v[x] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+    }
+  } else {
+    v[0] += __shfl_xor_sync(0xffffffffu, v[0], mask);
+  }
+}
+
+template <int D, int HPW, int WPB, int NST>
+__global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ? 3 : 1)
+    attn_splitk_kernel(const AttnParams p) {
+  using C = AttnCfg<D, HPW, WPB, NST>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint16_t* stages = reinterpret_cast<uint16_t*>(smem);
+  float* pbuf = reinterpret_cast<float*>(smem + C::OFF_P);
+  float* alph = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
+  int* flags = reinterpret_cast<int*>(smem + C::OFF_FLAGS);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
+  uint64_t* empty = full + NST;
+
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const PoolView& pool = p.pool;
+
+  // cached tokens of this sequence, clamped to what the table can hold
+  int ctx = p.seq_lens[b];
+  if (ctx < 0 || ctx / kT + 1 > p.max_blocks) {
+    if (threadIdx.x == 0 && s == 0 && g == 0) flag_error(pool.status, kErrCtxTooLong);
+    ctx = ctx < 0 ? 0 : min(ctx, p.max_blocks * kT);
+  }
+  const int nb = (ctx + kT - 1) / kT;
+  const int j0 = (int)((int64_t)nb * s / p.S);
+  const int j1 = (int)((int64_t)nb * (s + 1) / p.S);
+  const int n_local = j1 - j0;
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&full[i], 33);   // 32 producer lanes + 1 flag publish
+      mbar_init(&empty[i], WPB); // lane 0 of each warp of the consuming slot
+    }
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == C::NCW) {
+    // ------------------------------------------------------------------ producer
+    const int64_t rowbase = (int64_t)b * p.max_blocks;
+    for (int i = 0; i < n_local; ++i) {
+      const int st = i % NST;
+      const int k = i / NST;
+      if (k > 0 && !mbar_wait_bounded(&empty[st], (k - 1) & 1, pool.status)) break;
+      const int j = j0 + i;
+      const int tier = p.tier_map[rowbase + j];
+      const int64_t phys = p.table[rowbase + j];
+      const int ntok = min(kT, ctx - j * kT);
+      bool valid = true;
+      if (tier > 1) {
+        valid = false;
+        if (lane == 0) flag_error(pool.status, kErrBadTier);
+      } else if (phys < 0 || phys >= tier_blocks(pool, tier)) {
+        valid = false;
+        if (lane == 0) flag_error(pool.status, kErrBadBlock);
+      }
+      uint16_t* dst = stages + st * C::STAGE_ELEMS;
+      if (lane == 0) flags[st] = valid ? ntok : -1;
+      if (!valid) {
+        mbar_arrive(&full[st]);
+        if (lane == 0) mbar_arrive(&full[st]);
+        continue;
+      }
+      const uint16_t* kp = tier_base(pool, tier) + chunk_offset(pool, tier, p.layer, phys, 0, g);
+      const uint16_t* vp = tier_base(pool, tier) + chunk_offset(pool, tier, p.layer, phys, 1, g);
+      if (tier == DKV_TIER_HBM) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
+          mbar_arrive(&full[st]);
+          bulk_g2s(dst, kp, C::STAGE_BYTES / 2, &full[st]);
+          bulk_g2s(dst + kT * D, vp, C::STAGE_BYTES / 2, &full[st]);
+        } else {
+          mbar_arrive(&full[st]);
+        }
+      } else {
+        constexpr int PIECES = C::STAGE_BYTES / 16;  // 16-byte pieces per stage
+        constexpr int HALF = PIECES / 2;
+#pragma unroll
+        for (int c = 0; c < PIECES / 32; ++c) {
+          const int idx = c * 32 + lane;
+          const uint16_t* src = idx < HALF ? kp + idx * 8 : vp + (idx - HALF) * 8;
+          cp_async16(dst + idx * 8, src);
+        }
+        cp_async_arrive_noinc(&full[st]);
+        if (lane == 0) mbar_arrive(&full[st]);
+      }
+    }
+    cp_async_wait_all();
+    return;  // consumers below sync only among themselves (named barrier 1)
+  }
+
+  // -------------------------------------------------------------------- consumers
+  const int slot = warp / WPB, hq = warp % WPB;
+  const int tg = lane >> 3, dg = lane & 7;
+  const int hbase = g * C::G + hq * HPW;  // first global q head of this warp
+
+  float qreg[HPW][C::QCH][8];
+#pragma unroll
+  for (int h = 0; h < HPW; ++h)
+#pragma unroll
+    for (int hh = 0; hh < C::QCH; ++hh) {
+      const float4* src = reinterpret_cast<const float4*>(
+          p.qs + ((int64_t)b * p.Hq + hbase + h) * D + (dg + 8 * hh) * 8);
+      const float4 a = src[0], c = src[1];
+      qreg[h][hh][0] = a.x; qreg[h][hh][1] = a.y; qreg[h][hh][2] = a.z; qreg[h][hh][3] = a.w;
+      qreg[h][hh][4] = c.x; qreg[h][hh][5] = c.y; qreg[h][hh][6] = c.z; qreg[h][hh][7] = c.w;
+    }
+
+  float acc[HPW][C::DPL];
+#pragma unroll
+  for (int h = 0; h < HPW; ++h)
+#pragma unroll
+    for (int e = 0; e < C::DPL; ++e) acc[h][e] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;  // state of head h_lane (lane-group uniform m)
+  const int h_lane = dg >> (3 - C::LOGH);
+  const bool head_leader = tg == 0 && (dg & C::LOWMASK) == 0;
+  float* pb = pbuf + warp * kT * HPW;
+  float* al = alph + warp * HPW;
+
+  for (int i = slot; i < n_local; i += kSlots) {
+    const int st = i % NST;
+    if (!mbar_wait_bounded(&full[st], (i / NST) & 1, pool.status)) break;
+    const int ntok = flags[st];
+    if (ntok > 0) {
+      const uint16_t* Ks = stages + st * C::STAGE_ELEMS;
+      const uint16_t* Vs = Ks + kT * D;
+      // ---- partial scores: lane (tg, dg) covers tokens tg + 4 i4 and 16-byte key
+      // chunks dg + 8 hh (eight lanes read one 128-byte row segment: no bank conflicts)
+      float v[C::NV];
+#pragma unroll
+      for (int x = 0; x < C::NV; ++x) v[x] = 0.f;
+#pragma unroll
+      for (int i4 = 0; i4 < 4; ++i4) {
+        const int t = tg + 4 * i4;
+#pragma unroll
+        for (int hh = 0; hh < C::QCH; ++hh) {
+          const uint4 w = *reinterpret_cast<const uint4*>(Ks + t * D + (dg + 8 * hh) * 8);
+          const float kf[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
+                               bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+#pragma unroll
+          for (int h = 0; h < HPW; ++h)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[h * 4 + i4] = fmaf(qreg[h][hh][e], kf[e], v[h * 4 + i4]);
+        }
+      }
+      // ---- reduce-scatter over the 8 dg lanes (masks 4, 2, 1): value index h*4+i4
+      rs_level<C::NV>(v, (dg & 4) != 0, 4);
+      rs_level<(C::NV >= 2 ? C::NV / 2 : 1)>(v, (dg & 2) != 0, 2);
+      rs_level<(C::NV >= 4 ? C::NV / 4 : 1)>(v, (dg & 1) != 0, 1);
+      // lane now holds NR full scores of head h_lane
+      float sv[C::NR];
+      int tk[C::NR];
+      float bmax = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < C::NR; ++r) {
+        const int idx = C::NV >= 8 ? dg * C::NR + r : (dg >> 1);
+        tk[r] = tg + 4 * (idx & 3);
+        sv[r] = tk[r] < ntok ? v[r] : -INFINITY;
+        bmax = fmaxf(bmax, sv[r]);
+      }
+#pragma unroll
+      for (int mask = 1; mask <= C::LOWMASK; mask <<= 1)
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, mask));
+      bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 8));
+      bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, 16));
+      const float m_new = fmaxf(m_run, bmax);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = fast_exp2(m_run - m_use);
+      float psum = 0.f;
+#pragma unroll
+      for (int r = 0; r < C::NR; ++r) {
+        const float pr = fast_exp2(sv[r] - m_use);
+        if (C::NV >= 8 || (dg & 1) == 0) {
+          pb[tk[r] * HPW + h_lane] = pr;
+          psum += pr;
+        }
+      }
+      l_run = l_run * alpha + psum;
+      m_run = m_new;
+      if (head_leader) al[h_lane] = alpha;
+      __syncwarp();
+      // ---- P.V: lane owns value dims [lane*DPL, lane*DPL + DPL)
+      float a_h[HPW];
+#pragma unroll
+      for (int h = 0; h < HPW; ++h) a_h[h] = al[h];
+#pragma unroll
+      for (int h = 0; h < HPW; ++h)
+#pragma unroll
+        for (int e = 0; e < C::DPL; ++e) acc[h][e] *= a_h[h];
+      const int d0 = lane * C::DPL;
+#pragma unroll
+      for (int t = 0; t < kT; ++t) {
+        if (t < ntok) {
+          float vf[C::DPL];
+          if constexpr (C::DPL == 4) {
+            const uint2 w = *reinterpret_cast<const uint2*>(Vs + t * D + d0);
+            vf[0] = bf16lo(w.x); vf[1] = bf16hi(w.x); vf[2] = bf16lo(w.y); vf[3] = bf16hi(w.y);
+          } else {
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(Vs + t * D + d0);
+            vf[0] = bf16lo(w); vf[1] = bf16hi(w);
+          }
+          float pp[HPW];
+          if constexpr (HPW == 4) {
+            const float4 q4 = *reinterpret_cast<const float4*>(pb + t * 4);
+            pp[0] = q4.x; pp[1] = q4.y; pp[2] = q4.z; pp[3] = q4.w;
+          } else {
+#pragma unroll
+            for (int h = 0; h < HPW; ++h) pp[h] = pb[t * HPW + h];
+          }
+#pragma unroll
+          for (int h = 0; h < HPW; ++h)
+#pragma unroll
+            for (int e = 0; e < C::DPL; ++e) acc[h][e] = fmaf(pp[h], vf[e], acc[h][e]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+
+  // ---- per-warp totals of l, then merge the four slots through shared memory
+  float l_tot = l_run;
+#pragma unroll
+  for (int mask = 1; mask <= C::LOWMASK; mask <<= 1) l_tot += __shfl_xor_sync(0xffffffffu, l_tot, mask);
+  l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 8);
+  l_tot += __shfl_xor_sync(0xffffffffu, l_tot, 16);
+
+  named_bar_sync(1, C::NCW * 32);  // every slot is done reading the stage ring
+  float* macc = reinterpret_cast<float*>(smem);
+  float2* mml = reinterpret_cast<float2*>(smem + C::NCW * HPW * D * 4);
+#pragma unroll
+  for (int h = 0; h < HPW; ++h)
+#pragma unroll
+    for (int e = 0; e < C::DPL; ++e) macc[(warp * HPW + h) * D + lane * C::DPL + e] = acc[h][e];
+  if (head_leader) mml[warp * HPW + h_lane] = make_float2(m_run, l_tot);
+  named_bar_sync(1, C::NCW * 32);
+
+  for (int o = threadIdx.x; o < C::G * D; o += C::NCW * 32) {
+    const int hh = o / D, d = o % D;
+    const int wq = hh / HPW, h = hh % HPW;
+    float M = -INFINITY;
+#pragma unroll
+    for (int sl = 0; sl < kSlots; ++sl) M = fmaxf(M, mml[(sl * WPB + wq) * HPW + h].x);
+    float A = 0.f, Ls = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int sl = 0; sl < kSlots; ++sl) {
+        const float2 ml = mml[(sl * WPB + wq) * HPW + h];
+        const float w = fast_exp2(ml.x - M);
+        A = fmaf(macc[((sl * WPB + wq) * HPW + h) * D + d], w, A);
+        Ls = fmaf(ml.y, w, Ls);
+      }
+    }
+    const int64_t base = ((int64_t)b * p.Hq + g * C::G + hh) * p.S + s;
+    p.part_acc[base * D + d] = A;
+    if (d == 0) p.part_ml[base] = make_float2(M, Ls);
+  }
+}
+
+// ----------------------------------------------------------------------- combine
+
+// out[b][h] = (sum_s acc_s 2^(m_s-M) + v_new 2^(s_new-M)) / (sum_s l_s 2^(m_s-M) + 2^(s_new-M))
+// over the S split partials and the new token's (score s_new, value v_hat); bf16 RNE.
+template <int D>
+__global__ void __launch_bounds__(D) combine_kernel(int Hq, int Hkv, int S,
+                                                    const float2* __restrict__ ml,
+                                                    const float* __restrict__ acc,
+                                                    const float* __restrict__ snew,
+                                                    const float* __restrict__ vnew,
+                                                    uint16_t* __restrict__ out) {
+  const int hg = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+  const int g = hg / (Hq / Hkv);
+  const int64_t base = ((int64_t)b * Hq + hg) * S;
+  const float sn = snew[(int64_t)b * Hq + hg];
+  float M = sn;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, ml[base + s].x);
+  const float wn = exp2f(sn - M);
+  float L = wn;
+  float A = wn * vnew[((int64_t)b * Hkv + g) * D + d];
+  for (int s = 0; s < S; ++s) {
+    const float2 m = ml[base + s];
+    if (m.x != -INFINITY) {
+      const float w = exp2f(m.x - M);
+      L = fmaf(m.y, w, L);
+      A = fmaf(acc[(base + s) * D + d], w, A);
+    }
+  }
+  out[((int64_t)b * Hq + hg) * D + d] = f32_to_bf16_bits(A / L);
+}
+
+// ---------------------------------------------------------------------- launchers
+
+template <int D, int HPW, int WPB>
+static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
+  constexpr int NST = 8;
+  using C = AttnCfg<D, HPW, WPB, NST>;
+  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST>;
+  static bool attr_done = false;  // per instantiation
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return cuda_check(e, "attention: set smem attribute");
+    attr_done = true;
+  }
+  dim3 grid(p.S, Hkv, B);
+  fn<<<grid, C::THREADS, C::SMEM, st>>>(p);
+  return cuda_check(cudaGetLastError(), "attention launch");
+}
+
+int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, cudaStream_t st) {
+  if (D == 128) {
+    switch (G) {
+      case 1: return launch_attn_t<128, 1, 1>(p, B, Hkv, st);
+      case 2: return launch_attn_t<128, 2, 1>(p, B, Hkv, st);
+      case 4: return launch_attn_t<128, 4, 1>(p, B, Hkv, st);
+      case 8: return launch_attn_t<128, 4, 2>(p, B, Hkv, st);
+    }
+  } else if (D == 64) {
+    switch (G) {
+      case 1: return launch_attn_t<64, 1, 1>(p, B, Hkv, st);
+      case 2: return launch_attn_t<64, 2, 1>(p, B, Hkv, st);
+      case 4: return launch_attn_t<64, 4, 1>(p, B, Hkv, st);
+      case 8: return launch_attn_t<64, 4, 2>(p, B, Hkv, st);
+    }
+  }
+  return set_error(DKV_ERR_UNSUPPORTED, "attention: unsupported D=%d G=%d", D, G);
+}
+
+int launch_combine(int B, int Hq, int Hkv, int D, int S, const float2* ml, const float* acc,
+                   const float* snew, const float* vnew, uint16_t* out, cudaStream_t st) {
+  dim3 grid(Hq, B);
+  if (D == 128)
+    combine_kernel<128><<<grid, 128, 0, st>>>(Hq, Hkv, S, ml, acc, snew, vnew, out);
+  else
+    combine_kernel<64><<<grid, 64, 0, st>>>(Hq, Hkv, S, ml, acc, snew, vnew, out);
+  return cuda_check(cudaGetLastError(), "combine launch");
+}
+
+}  // namespace dkv

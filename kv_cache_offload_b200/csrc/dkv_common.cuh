@@ -1,0 +1,158 @@
+// Shared device-side helpers for libdkv (sm_100a): pool view, error bits, mbarrier,
+// bulk-copy and cp.async wrappers, bounded waits.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/dkv.h"
+
+namespace dkv {
+
+// Status-word bits set by kernels (never trap; skip and flag instead).
+enum : int {
+  kErrBadTier = 1,
+  kErrBadBlock = 2,
+  kErrCtxTooLong = 4,
+  kErrTimeout = 8,
+};
+
+// What a kernel needs to address the pool.
+struct PoolView {
+  uint16_t* tier[2];     // device-accessible bases (HBM, host alias)
+  int64_t blocks[2];     // physical blocks per tier
+  int32_t L, Hkv, D, T;
+  int32_t layout;        // DKV_LAYOUT_*
+  int* status;           // device status word
+};
+
+// Element offset of the [T][D] chunk (layer, phys, kv, g) inside a tier.
+__host__ __device__ __forceinline__ int64_t chunk_offset(const PoolView& p, int tier, int layer,
+                                                         int64_t phys, int kv, int g) {
+  int64_t c;
+  if (p.layout == DKV_LAYOUT_LAYER_FIRST)
+    c = (((int64_t)layer * (tier ? p.blocks[1] : p.blocks[0]) + phys) * 2 + kv) * p.Hkv + g;
+  else
+    c = (((int64_t)phys * p.L + layer) * 2 + kv) * p.Hkv + g;
+  return c * (int64_t)p.T * p.D;
+}
+
+// Tier base / size selected without dynamic indexing into the by-value struct (which
+// would put the struct in local memory).
+__host__ __device__ __forceinline__ uint16_t* tier_base(const PoolView& p, int tier) {
+  return tier ? p.tier[1] : p.tier[0];
+}
+__host__ __device__ __forceinline__ int64_t tier_blocks(const PoolView& p, int tier) {
+  return tier ? p.blocks[1] : p.blocks[0];
+}
+
+__device__ __forceinline__ void flag_error(int* status, int bits) {
+  if (status) atomicOr(status, bits);
+}
+
+// ------------------------------------------------------------------ shared memory
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for the phase with `parity` to complete, giving up after `limit_ns` of wall time.
+// Returns false (and flags kErrTimeout) on give-up. Never spins forever.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* status,
+                                                  uint64_t limit_ns = 4000000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u && globaltimer_ns() - t0 > limit_ns) {
+      flag_error(status, kErrTimeout);
+      return false;
+    }
+  }
+}
+
+// ------------------------------------------------------------------- bulk copies
+
+// 1-D bulk copy global -> shared (TMA engine), completing `bytes` on `bar`.
+// Requires 16-byte aligned addresses and bytes % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(dst_smem)),
+      "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared through the LSU (works for mapped host memory).
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src)
+               : "memory");
+}
+
+// Arrive on `bar` once all of this thread's prior cp.async copies have landed; the arrival
+// counts against the barrier's initial count (no pending-count increment).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// Named barrier among `nthreads` threads (multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ------------------------------------------------------------------ conversions
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+}  // namespace dkv

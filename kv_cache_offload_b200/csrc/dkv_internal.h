@@ -1,0 +1,77 @@
+// Host-side internals shared by the libdkv translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dkv.h"
+#include "dkv_common.cuh"
+
+struct dkv_pool {
+  dkv_pool_config cfg;
+  int device;
+  int num_sms;
+  uint16_t* hbm;
+  size_t hbm_bytes;
+  bool own_hbm;
+  uint16_t* host_h;   // host-side address of the host tier
+  uint16_t* host_d;   // device alias of the host tier
+  size_t host_bytes;
+  int* d_status;
+  dkv_tuning tuning;
+
+  dkv::PoolView view() const {
+    dkv::PoolView v;
+    v.tier[0] = hbm;
+    v.tier[1] = host_d;
+    v.blocks[0] = cfg.hbm_blocks;
+    v.blocks[1] = cfg.host_blocks;
+    v.L = cfg.num_layers;
+    v.Hkv = cfg.num_kv_heads;
+    v.D = cfg.head_dim;
+    v.T = cfg.block_tokens;
+    v.layout = cfg.layout;
+    v.status = d_status;
+    return v;
+  }
+};
+
+namespace dkv {
+
+int set_error(int code, const char* fmt, ...);
+int cuda_check(cudaError_t e, const char* what);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Arguments of the split-K attention kernel.
+struct AttnParams {
+  PoolView pool;
+  int layer;
+  const int32_t* table;
+  const int32_t* seq_lens;
+  const uint8_t* tier_map;
+  int max_blocks;
+  int Hq;
+  int S;
+  const float* qs;   // [B][Hq][D], scaled by log2(e)/sqrt(D)
+  float2* part_ml;   // [B][Hq][S] (m, l)
+  float* part_acc;   // [B][Hq][S][D]
+};
+
+int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, cudaStream_t st);
+int launch_combine(int B, int Hq, int Hkv, int D, int S, const float2* ml, const float* acc,
+                   const float* snew, const float* vnew, uint16_t* out, cudaStream_t st);
+
+// Workspace carve-up of one decode step (all offsets 256-byte aligned).
+struct DecodeWs {
+  int B, Hq, Hkv, D, rows, S, G, max_blocks, hidden, proj_splits;
+  size_t off_proj_acc, off_proj_cnt, off_qs, off_snew, off_vnew, off_ml, off_acc, total;
+};
+
+// Fills `w` for a shape; returns DKV_OK or an error (unsupported shape).
+int decode_ws_layout(const dkv_pool* pool, int B, int max_blocks, int Hq, int hidden,
+                     DecodeWs* w);
+
+}  // namespace dkv

@@ -1,0 +1,184 @@
+"""Parity of the CUDA decode step (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as WL
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import kv_cache_offload_b200 as dkv
+    import dkv_testlib as TL
+else:  # collected on CPU-only hosts, never run
+    dkv = TL = None
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from kv_cache_offload_b200.build import build
+    build()
+
+
+def _run_and_check(cfg, seed=0, layout=0, layer=None, attn_splits=0, seq_lens=None, host_flags=0):
+    inp = WL.make_decode_inputs(cfg, seed=seed, pool_layout=layout, seq_lens=seq_lens)
+    layer = cfg.layers - 1 if layer is None else layer
+    ctx = TL.make_pool(inp, host_flags=host_flags)
+    try:
+        out = TL.run_step(ctx, layer=layer, attn_splits=attn_splits)
+        ores = TL.oracle_step(inp, layer=layer)
+        errs = TL.assert_out_close(out, ores["out"], cfg.name)
+        TL.check_cache(ctx, ores, layer=layer)
+        return out, ores, errs
+    finally:
+        ctx.close()
+
+
+def test_tiny_config_all_host():
+    _run_and_check(WL.CONFIGS["tiny"])
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(8, 2, 128), (8, 8, 128), (4, 2, 128), (16, 2, 128),
+                                      (8, 2, 64), (8, 8, 64), (4, 2, 64), (16, 2, 64)])
+def test_group_sizes_and_head_dims(Hq, Hkv, D):
+    cfg = WL.small_config(Hq=Hq, Hkv=Hkv, D=D, H=256 if D == 64 else 384)
+    _run_and_check(cfg)
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_ragged_lengths_both_tiers_both_layouts(layout):
+    cfg = WL.small_config(B=7, layers=3)
+    _run_and_check(cfg, layout=layout, layer=1, seq_lens=[0, 1, 15, 16, 17, 100, 257])
+
+
+@pytest.mark.parametrize("splits", [1, 2, 5, 64])
+def test_split_counts(splits):
+    cfg = WL.small_config(B=2, ctx_range=(300, 400))
+    _run_and_check(cfg, attn_splits=splits)
+
+
+def test_split_invariance_close():
+    cfg = WL.small_config(B=2, ctx_range=(500, 700), host_prob=0.3)
+    o1, _, _ = _run_and_check(cfg, attn_splits=1)
+    o2, _, _ = _run_and_check(cfg, attn_splits=13)
+    d = (o1.float() - o2.float()).abs().max().item()
+    assert d <= 2 * 2.0 ** -8 * max(o1.float().abs().max().item(), 1e-3)
+
+
+def test_batch_32_and_write_combined_host():
+    cfg = WL.small_config(B=32, H=256, Hq=8, Hkv=8, D=64, ctx_range=(1, 90), layers=1)
+    _run_and_check(cfg, host_flags=dkv.DKV_HOST_WRITE_COMBINED)
+
+
+def test_step_is_repeatable():
+    cfg = WL.small_config(B=3)
+    inp = WL.make_decode_inputs(cfg)
+    ctx = TL.make_pool(inp)
+    try:
+        a = TL.run_step(ctx, layer=1)
+        b = TL.run_step(ctx, layer=1)
+        # the same inputs give the same result up to the order of the projection's fp32
+        # split-K reduction (one bf16 ulp at most)
+        d = (a.float() - b.float()).abs()
+        assert (d <= 2.0 ** -7 * a.float().abs().clamp_min(2.0 ** -20)).all()
+    finally:
+        ctx.close()
+
+
+def test_bad_table_entries_are_flagged_not_fatal():
+    cfg = WL.small_config(B=2, ctx_range=(40, 60), host_prob=0.5)
+    inp = WL.make_decode_inputs(cfg)
+    ctx = TL.make_pool(inp)
+    try:
+        x, W = inp.x.cuda(), inp.W.cuda()
+        out = torch.empty((cfg.B, cfg.Hq * cfg.D), dtype=torch.bfloat16, device="cuda")
+        nws = dkv.dkv_decode_workspace_bytes(ctx.pool, cfg.B, ctx.table.shape[1], cfg.Hq, cfg.H)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        for mutate in ("tier", "block", "ctx"):
+            table, tmap, lens = ctx.table.clone(), ctx.tier_map.clone(), ctx.seq_lens.clone()
+            if mutate == "tier":
+                tmap[0, 1] = 7
+            elif mutate == "block":
+                table[1, 0] = 1 << 30
+            else:
+                lens[0] = table.shape[1] * cfg.T + 5
+            dkv.dkv_decode_step(ctx.pool, 1, x, W, table, lens, tmap, cfg.Hq, cfg.theta, out, ws)
+            assert dkv.dkv_check(ctx.pool) == dkv.DKV_ERR_BAD_TABLE, mutate
+        # the pool is still usable and clean afterwards
+        assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
+    finally:
+        ctx.close()
+
+
+def test_argument_errors():
+    cfg = WL.small_config(B=2)
+    inp = WL.make_decode_inputs(cfg)
+    ctx = TL.make_pool(inp)
+    try:
+        with pytest.raises(dkv.DkvError):
+            dkv.dkv_decode_workspace_bytes(ctx.pool, 33, ctx.table.shape[1], cfg.Hq, cfg.H)
+        with pytest.raises(dkv.DkvError):
+            dkv.dkv_decode_workspace_bytes(ctx.pool, 2, ctx.table.shape[1], 6, cfg.H)  # G = 3
+        nws = dkv.dkv_decode_workspace_bytes(ctx.pool, 2, ctx.table.shape[1], cfg.Hq, cfg.H)
+        ws = torch.empty(nws - 256, dtype=torch.uint8, device="cuda")
+        out = torch.empty((2, cfg.Hq * cfg.D), dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(dkv.DkvError):
+            dkv.dkv_decode_step(ctx.pool, 0, inp.x.cuda(), inp.W.cuda(), ctx.table, ctx.seq_lens,
+                                ctx.tier_map, cfg.Hq, cfg.theta, out, ws)
+    finally:
+        ctx.close()
+
+
+def test_append_kv_places_tokens_bit_exact():
+    cfg = WL.small_config(B=3, ctx_range=(5, 40), layers=2)
+    inp = WL.make_decode_inputs(cfg)
+    ctx = TL.make_pool(inp)
+    try:
+        n = 9
+        lens = [max(0, c - n) for c in inp.layout.seq_lens]  # positions that exist in the table
+        k = WL.randn_bf16((cfg.B, n, cfg.Hkv, cfg.D), 77)
+        v = WL.randn_bf16((cfg.B, n, cfg.Hkv, cfg.D), 78)
+        lens_d = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        dkv.dkv_append_kv(ctx.pool, 1, k.cuda(), v.cuda(), ctx.table, lens_d, ctx.tier_map)
+        assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
+        exp = [WL.bf16_bits(inp.hbm).copy(), WL.bf16_bits(inp.host).copy()]
+        kb, vb = WL.bf16_bits(k), WL.bf16_bits(v)
+        for b in range(cfg.B):
+            for t in range(n):
+                pos = lens[b] + t
+                j, slot = divmod(pos, cfg.T)
+                tier = int(inp.layout.tier_map[b, j]); phys = int(inp.layout.block_table[b, j])
+                exp[tier][1, phys, 0, :, slot] = kb[b, t]
+                exp[tier][1, phys, 1, :, slot] = vb[b, t]
+        got = [ctx.hbm.cpu().view(torch.int16).numpy().view(np.uint16).reshape(inp.hbm.shape),
+               ctx.host.numpy().view(np.uint16).reshape(inp.host.shape)]
+        assert np.array_equal(got[0], exp[0]) and np.array_equal(got[1], exp[1])
+    finally:
+        ctx.close()
+
+
+@pytest.mark.parametrize("src_tier", [0, 1])
+def test_layout_conversion_bit_exact(src_tier):
+    from oracle import dkv_oracle as O
+    cfg = WL.small_config(B=4, layers=5, ctx_range=(30, 200), host_prob=0.5)
+    for layout in (0, 1):
+        inp = WL.make_decode_inputs(cfg, pool_layout=layout)
+        ctx = TL.make_pool(inp)
+        try:
+            src = (inp.hbm, inp.host)[src_tier]
+            dst = torch.empty(src.numel(), dtype=torch.bfloat16, device="cuda")
+            dkv.dkv_convert_layout(ctx.pool, src_tier, dst)
+            torch.cuda.synchronize()
+            bits = WL.bf16_bits(src)
+            exp = O.layer_first_to_page_first(bits) if layout == 0 else O.page_first_to_layer_first(bits)
+            got = dst.cpu().view(torch.int16).numpy().view(np.uint16).reshape(exp.shape)
+            assert np.array_equal(got, exp)
+            # and back again with the raw-buffer entry point
+            back = torch.empty_like(dst)
+            chunk = 2 * cfg.Hkv * cfg.T * cfg.D * 2
+            nblk = src.shape[1] if layout == 0 else src.shape[0]
+            dkv.dkv_permute_layout(dst, back, 1 - layout, cfg.layers, nblk, chunk)
+            torch.cuda.synchronize()
+            assert np.array_equal(back.cpu().view(torch.int16).numpy().view(np.uint16), bits.reshape(-1))
+        finally:
+            ctx.close()
