@@ -64,10 +64,31 @@ int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, cudaStre
 int launch_combine(int B, int Hq, int Hkv, int D, int S, const float2* ml, const float* acc,
                    const float* snew, const float* vnew, uint16_t* out, cudaStream_t st);
 
+// Arguments of one projection launch (see dkv_projection.cu).
+struct ProjArgs {
+  PoolView pool;
+  int layer;
+  const uint16_t* x;
+  const uint16_t* W;
+  const int32_t* table;
+  const int32_t* seq_lens;
+  const uint8_t* tier_map;
+  int max_blocks;
+  int B, H, Hq, Hkv, D;
+  double theta;
+  float qscale;   // log2(e) / sqrt(D)
+  float* qs;      // [B][Hq][D]
+  float* snew;    // [B][Hq]
+  float* vnew;    // [B][Hkv][D]
+  int cluster;    // cluster size request (0 = automatic)
+};
+
+int launch_projection(const ProjArgs& a, cudaStream_t st);
+
 // Workspace carve-up of one decode step (all offsets 256-byte aligned).
 struct DecodeWs {
-  int B, Hq, Hkv, D, rows, S, G, max_blocks, hidden, proj_splits;
-  size_t off_proj_acc, off_proj_cnt, off_qs, off_snew, off_vnew, off_ml, off_acc, total;
+  int B, Hq, Hkv, D, rows, S, G, max_blocks, hidden;
+  size_t off_qs, off_snew, off_vnew, off_ml, off_acc, total;
 };
 
 // Fills `w` for a shape; returns DKV_OK or an error (unsupported shape).
