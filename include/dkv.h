@@ -168,6 +168,32 @@ int dkv_decode_attend(dkv_pool* pool, int layer, const int32_t* block_table,
 int dkv_decode_combine(dkv_pool* pool, int B, int max_blocks, int hidden, int num_q_heads,
                        uint16_t* out, void* workspace, size_t ws_bytes, void* stream);
 
+/*
+ * dkv_decode_step without a caller workspace, for callers that cannot allocate device
+ * memory: a serving loop whose device memory is all reserved up front by its own allocator
+ * (a cudaMalloc there fails or fragments that reservation), a latency-critical loop that
+ * cannot take cudaMalloc's implicit synchronisation, or a plain C host with no device
+ * allocator. The paper has no counterpart to this call; it is a deployment convenience.
+ * Same arguments and results as dkv_decode_step; the workspace is a fixed array of
+ * dkv_decode_static_workspace_capacity() bytes (16 MiB) in the library's own device memory,
+ * which every GPU that loads the library holds until the process exits. The call allocates
+ * nothing (no cudaMalloc/cudaFree, no allocating library routine).
+ *  - The first call on a device looks up that device's array address (cudaGetSymbolAddress
+ *    with the device current); make that first call before any stream capture.
+ *  - Shapes whose workspace (dkv_decode_workspace_bytes) exceeds the capacity are rejected
+ *    with DKV_ERR_CAPACITY and nothing is launched.
+ *  - Every call shares the one array per device and it keeps the last call's contents;
+ *    nothing in it needs to start at zero (each step writes every word it later reads).
+ *    Calls whose execution overlaps on the GPU (different streams, no ordering) race on it.
+ */
+int dkv_decode_step_static(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t* Wqkv,
+                           const int32_t* block_table, const int32_t* seq_lens,
+                           const uint8_t* tier_map, int B, int max_blocks, int hidden,
+                           int num_q_heads, float rope_theta, uint16_t* out, void* stream);
+
+/* Size in bytes of the per-device static workspace dkv_decode_step_static uses. */
+size_t dkv_decode_static_workspace_capacity(void);
+
 /* The attention split-K factor dkv_decode_step uses for this shape (after tuning). */
 int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 

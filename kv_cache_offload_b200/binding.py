@@ -69,6 +69,8 @@ _SIGS = {
     "dkv_decode_attend": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
     "dkv_decode_combine": (_I, [_P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dkv_decode_attn_splits": (_I, [_P, _I, _I, _I]),
+    "dkv_decode_step_static": (_I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]),
+    "dkv_decode_static_workspace_capacity": (_SZ, []),
     "dkv_permute_layout": (_I, [_P, _P, _I, _I, _I64, _I64, _P]),
     "dkv_convert_layout": (_I, [_P, _I, _P, _SZ, _P]),
     "dkv_check": (_I, [_P, _P]),
@@ -228,6 +230,22 @@ def dkv_decode_step(pool: int, layer: int, x: torch.Tensor, Wqkv: torch.Tensor,
                                _ptr(tier_map), B, block_table.shape[1], H, num_q_heads,
                                float(rope_theta), _ptr(out), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dkv_decode_step_static(pool: int, layer: int, x: torch.Tensor, Wqkv: torch.Tensor,
+                           block_table: torch.Tensor, seq_lens: torch.Tensor, tier_map: torch.Tensor,
+                           num_q_heads: int, rope_theta: float, out: torch.Tensor, stream=None):
+    """dkv_decode_step with the library's fixed per-device workspace: allocates nothing."""
+    _decode_checks(x, Wqkv, block_table, seq_lens, tier_map)
+    _need(out, torch.bfloat16, "out")
+    B, H = x.shape
+    _chk(lib().dkv_decode_step_static(pool, layer, _ptr(x), _ptr(Wqkv), _ptr(block_table), _ptr(seq_lens),
+                                      _ptr(tier_map), B, block_table.shape[1], H, num_q_heads,
+                                      float(rope_theta), _ptr(out), _stream(stream)))
+
+
+def dkv_decode_static_workspace_capacity() -> int:
+    return lib().dkv_decode_static_workspace_capacity()
 
 
 def dkv_decode_project(pool, layer, x, Wqkv, block_table, seq_lens, tier_map, num_q_heads,
