@@ -37,14 +37,17 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="dkv", choices=["dkv", "reference"])
     ap.add_argument("--config", default="8b_hbm", choices=sorted(WL.CONFIGS))
     ap.add_argument("--attn-splits", type=int, default=0)
     ap.add_argument("--proj-splits", type=int, default=0)
     ap.add_argument("--host-flags", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
+    ap.add_argument("--profile", action="store_true",
+                    help="warm-up + timed steps only (no clock pre-roll, e2e or CPU baseline): for ncu")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
     return ap.parse_args()
 
@@ -201,10 +204,14 @@ class Workload:
         self.new_kv_bytes = cfg.B * cfg.Hkv * cfg.D * 2 * 2
         self.splits = dkv.dkv_decode_attn_splits(self.pool, cfg.B, lay.max_blocks, cfg.Hq)
 
-    def set_tuning(self, attn_splits=0, proj_splits=0):
-        self.dkv.dkv_pool_set_tuning(self.pool, attn_splits=attn_splits, proj_splits=proj_splits)
-        self.splits = self.dkv.dkv_decode_attn_splits(self.pool, self.cfg.B, self.lay.max_blocks,
-                                                      self.cfg.Hq)
+    def set_tuning(self, attn_splits=0, proj_splits=0, **kw):
+        c = self.cfg
+        self.dkv.dkv_pool_set_tuning(self.pool, attn_splits=attn_splits, proj_splits=proj_splits, **kw)
+        self.splits = self.dkv.dkv_decode_attn_splits(self.pool, c.B, self.lay.max_blocks, c.Hq)
+        n = self.dkv.dkv_decode_workspace_bytes(self.pool, c.B, self.lay.max_blocks, c.Hq, c.H)
+        if n > self.nws:
+            self.nws = n
+            self.ws = torch.empty(n, dtype=torch.uint8, device=self.ws.device)
 
     def step(self):
         c = self.cfg
@@ -212,15 +219,15 @@ class Workload:
                                  c.theta, self.out, self.ws)
 
     def step_timed_stages(self, ev):
+        """The same step as step(), with events between its two launches."""
         c, d = self.cfg, self.dkv
         ev[0].record()
         d.dkv_decode_project(self.pool, 0, self.x, self.W, self.table, self.lens, self.tmap, c.Hq,
                              c.theta, self.ws)
         ev[1].record()
-        d.dkv_decode_attend(self.pool, 0, self.table, self.lens, self.tmap, c.H, c.Hq, self.ws)
+        d.dkv_decode_attend(self.pool, 0, self.table, self.lens, self.tmap, c.H, c.Hq, self.ws,
+                            out=self.out)
         ev[2].record()
-        d.dkv_decode_combine(self.pool, c.B, self.lay.max_blocks, c.H, c.Hq, self.out, self.ws)
-        ev[3].record()
 
     def close(self):
         if self.pool:
@@ -348,6 +355,9 @@ def main():
     import kv_cache_offload_b200 as dkv
 
     cfg = WL.CONFIGS[args.config]
+    if args.batch:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, B=args.batch)
     wl = Workload(cfg, seed=rank, host_flags=args.host_flags)
     wl.set_tuning(args.attn_splits, args.proj_splits)
 
@@ -359,29 +369,50 @@ def main():
     for _ in range(args.warmup):
         wl.step()
     assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
+    if args.profile:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            wl.step()
+        b.record()
+        b.synchronize()
+        assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
+        if rank == 0:
+            print(json.dumps({"profile_run": cfg.name, "B": cfg.B, "attn_splits": wl.splits,
+                              "ms_per_step": a.elapsed_time(b) / args.steps}), flush=True)
+        wl.close()
+        return
 
-    # ---- value: K back-to-back steps, inputs resident in HBM / host tier
+    # ---- value: K back-to-back steps, inputs resident in HBM / host tier. The clock
+    # sampler (200 ms period) starts first and the GPU is kept busy with untimed steps for
+    # ~0.6 s so that samples are taken under the same load as the timed region.
     clocks = ClockSampler(local)
     barrier()
     clocks.start()
+    t_end = time.perf_counter() + 0.6
+    while time.perf_counter() < t_end:
+        for _ in range(8):
+            wl.step()
+        torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(args.steps):
         wl.step()
     e1.record()
     barrier()
+    time.sleep(0.25)
     clk = clocks.stop()
     t_ms = e0.elapsed_time(e1)
     assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
 
     # ---- per-stage durations (same steps with events between the three launches)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier()
     for i in range(args.steps):
         wl.step_timed_stages(evs[i])
     barrier()
     stage_ms = [sum(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)) / args.steps
-                for k in range(3)]
+                for k in range(2)]
 
     # ---- e2e: host buffers in, result out, through the public API
     xh = wl.x.cpu().pin_memory()
@@ -436,14 +467,14 @@ def main():
                    "parallelism": "replicas x%d" % world, "attn_splits": wl.splits,
                    "l2": "inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)},
         "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
-        "stage_ms": {"project": stage_ms[0], "attend": stage_ms[1], "combine": stage_ms[2]},
+        "stage_ms": {"project": stage_ms[0], "attend_and_combine": stage_ms[1]},
         "roofline": {"bound": "hbm" if not wl.kv_host_bytes else "host_link", "kernel": "attn_splitk_kernel",
                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "peak_source": peak_kind,
                      "traffic": profiled_traffic(cfg.name),
                      "algorithmic_bytes_per_launch": wl.kv_bytes},
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
     if host_info:

@@ -79,8 +79,11 @@ typedef struct dkv_pool_config {
 /* Launch tunables; 0 means "choose automatically". */
 typedef struct dkv_tuning {
   int32_t attn_splits;   /* split-K factor of the attention grid (per sequence, kv head) */
-  int32_t proj_splits;   /* split factor of the projection's reduction dimension */
-  int32_t reserved[6];
+  int32_t proj_splits;   /* cluster size of the projection (its reduction split), <= 16 */
+  int32_t attn_variant;  /* attention kernel shape for G = 4: 0 default, 1 deeper ring,
+                            2 two warps per block, 3 both */
+  int32_t attn_lsu_hbm;  /* 1: load HBM-tier blocks with 16-byte cp.async, not bulk copies */
+  int32_t reserved[4];
 } dkv_tuning;
 
 /*
@@ -149,12 +152,15 @@ int dkv_decode_step(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t
                     size_t ws_bytes, void* stream);
 
 /*
- * The three stages of dkv_decode_step as separate calls, with the same arguments and the
- * same workspace (for timing each stage). dkv_decode_step == project; attend; combine.
- *   project: projection, RoPE, the single cache write, the new token's partial softmax
- *            state (score and value), q for the attention — all into the workspace.
- *   attend:  split-K partial softmax states over the cached blocks of both tiers.
- *   combine: merges the partial states and the new token's into out (bf16).
+ * The stages of dkv_decode_step as separate calls, with the same arguments and the same
+ * workspace (for timing each stage). dkv_decode_step == project; attend(out).
+ *   project: projection, RoPE, the single cache write of k_hat / v_hat, and q, k_hat,
+ *            v_hat (fp32) for the attention — into the workspace.
+ *   attend:  split-K partial softmax states over the cached blocks of both tiers; with
+ *            out != NULL the last split of each (sequence, kv head) also merges the
+ *            partial states with the new token's term (score q . k_hat, value v_hat) into
+ *            out (the combine, fused).
+ *   combine: the merge as its own kernel, for attend(out = NULL).
  */
 int dkv_decode_project(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t* Wqkv,
                        const int32_t* block_table, const int32_t* seq_lens,
@@ -163,8 +169,8 @@ int dkv_decode_project(dkv_pool* pool, int layer, const uint16_t* x, const uint1
                        void* stream);
 int dkv_decode_attend(dkv_pool* pool, int layer, const int32_t* block_table,
                       const int32_t* seq_lens, const uint8_t* tier_map, int B,
-                      int max_blocks, int hidden, int num_q_heads, void* workspace,
-                      size_t ws_bytes, void* stream);
+                      int max_blocks, int hidden, int num_q_heads, uint16_t* out,
+                      void* workspace, size_t ws_bytes, void* stream);
 int dkv_decode_combine(dkv_pool* pool, int B, int max_blocks, int hidden, int num_q_heads,
                        uint16_t* out, void* workspace, size_t ws_bytes, void* stream);
 

@@ -48,7 +48,8 @@ class dkv_pool_config(ctypes.Structure):
 
 class dkv_tuning(ctypes.Structure):
     _fields_ = [("attn_splits", ctypes.c_int32), ("proj_splits", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 6)]
+                ("attn_variant", ctypes.c_int32), ("attn_lsu_hbm", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 4)]
 
 
 _P = ctypes.c_void_p
@@ -66,7 +67,7 @@ _SIGS = {
     "dkv_decode_workspace_bytes": (_SZ, [_P, _I, _I, _I, _I]),
     "dkv_decode_step": (_I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P, _SZ, _P]),
     "dkv_decode_project": (_I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _SZ, _P]),
-    "dkv_decode_attend": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "dkv_decode_attend": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dkv_decode_combine": (_I, [_P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dkv_decode_attn_splits": (_I, [_P, _I, _I, _I]),
     "dkv_decode_step_static": (_I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]),
@@ -167,8 +168,9 @@ def dkv_pool_tier_ptr(pool: int, tier: int):
     return d.value, h.value, n.value
 
 
-def dkv_pool_set_tuning(pool: int, attn_splits: int = 0, proj_splits: int = 0):
-    t = dkv_tuning(attn_splits, proj_splits)
+def dkv_pool_set_tuning(pool: int, attn_splits: int = 0, proj_splits: int = 0,
+                        attn_variant: int = 0, attn_lsu_hbm: int = 0):
+    t = dkv_tuning(attn_splits, proj_splits, attn_variant, attn_lsu_hbm)
     _chk(lib().dkv_pool_set_tuning(pool, ctypes.byref(t)))
 
 
@@ -259,10 +261,13 @@ def dkv_decode_project(pool, layer, x, Wqkv, block_table, seq_lens, tier_map, nu
 
 
 def dkv_decode_attend(pool, layer, block_table, seq_lens, tier_map, hidden, num_q_heads,
-                      workspace, stream=None):
+                      workspace, out=None, stream=None):
+    """Split-K attention; with `out` the combine is fused (else call dkv_decode_combine)."""
     B = block_table.shape[0]
+    if out is not None:
+        _need(out, torch.bfloat16, "out")
     _chk(lib().dkv_decode_attend(pool, layer, _ptr(block_table), _ptr(seq_lens), _ptr(tier_map), B,
-                                 block_table.shape[1], hidden, num_q_heads, _ptr(workspace),
+                                 block_table.shape[1], hidden, num_q_heads, _ptr(out), _ptr(workspace),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
 
 

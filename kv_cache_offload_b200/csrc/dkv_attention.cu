@@ -43,7 +43,7 @@ struct AttnCfg {
   static constexpr int LOWMASK = (1 << (3 - LOGH)) - 1;  // dg bits shared by one head
   static constexpr int NR = NV >= 8 ? NV / 8 : 1;        // scores per lane after reduction
   static constexpr int OFF_P = NST * STAGE_BYTES;
-  static constexpr int OFF_ALPHA = OFF_P + NCW * kT * HPW * 4;
+  static constexpr int OFF_ALPHA = OFF_P + NCW * kT * HPW * 8;
   static constexpr int OFF_FLAGS = OFF_ALPHA + NCW * HPW * 4;
   static constexpr int OFF_BARS = (OFF_FLAGS + NST * 4 + 7) / 8 * 8;
   static constexpr int SMEM = OFF_BARS + 2 * NST * 8;
@@ -56,6 +56,39 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Merge the S split states of one (b, q head) output element with the new token's term:
+// M = max(s_new, m_s), L = 2^(s_new-M) + sum l_s 2^(m_s-M),
+// o = (v_new 2^(s_new-M) + sum acc_s 2^(m_s-M)) / L. Splits are read in index order.
+__device__ __forceinline__ float combine_value(const float2* __restrict__ ml, const float* __restrict__ acc,
+                                               int S, int64_t base, int D, int d, float sn, float vn) {
+  float M = sn;
+  for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(ml + base + s).x);
+  const float wn = exp2f(sn - M);
+  float L = wn;
+  float A = wn * vn;
+  for (int s = 0; s < S; ++s) {
+    const float2 m = __ldcg(ml + base + s);
+    if (m.x != -INFINITY) {
+      const float w = exp2f(m.x - M);
+      L = fmaf(m.y, w, L);
+      A = fmaf(__ldcg(acc + (base + s) * D + d), w, A);
+    }
+  }
+  return A / L;
+}
+
+// The new token's score s_new = q . k_hat (log2 domain: q is pre-scaled), computed by one
+// full warp in a fixed order (lane l sums dims l, l+32, ...; then a butterfly), so the
+// fused and the standalone combine produce identical bits.
+__device__ __forceinline__ float new_token_score(const float* __restrict__ q, const float* __restrict__ k, int D,
+                                                 int lane) {
+  float s = 0.f;
+  for (int d = lane; d < D; d += 32) s = fmaf(q[d], k[d], s);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return s;
 }
 
 // One level of a warp reduce-scatter: lanes with `up` keep the upper half of the N live
@@ -74,13 +107,13 @@ __device__ __forceinline__ void rs_level(float* v, bool up, int mask) {
   }
 }
 
-template <int D, int HPW, int WPB, int NST>
-__global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ? 3 : 1)
+template <int D, int HPW, int WPB, int NST, int MINB>
+__global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
     attn_splitk_kernel(const AttnParams p) {
   using C = AttnCfg<D, HPW, WPB, NST>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* stages = reinterpret_cast<uint16_t*>(smem);
-  float* pbuf = reinterpret_cast<float*>(smem + C::OFF_P);
+  float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
   float* alph = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
   int* flags = reinterpret_cast<int*>(smem + C::OFF_FLAGS);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
@@ -113,14 +146,24 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ?
 
   if (warp == C::NCW) {
     // ------------------------------------------------------------------ producer
+    // Table entries are fetched 32 blocks at a time (lane l holds block base + l) and
+    // broadcast by shuffle, so no dependent global load sits on the per-block path.
     const int64_t rowbase = (int64_t)b * p.max_blocks;
+    int pf_tier = 0, pf_phys = 0;
     for (int i = 0; i < n_local; ++i) {
+      if ((i & 31) == 0) {
+        const int j = j0 + i + lane;
+        if (j < j1) {
+          pf_tier = p.tier_map[rowbase + j];
+          pf_phys = p.table[rowbase + j];
+        }
+      }
       const int st = i % NST;
       const int k = i / NST;
       if (k > 0 && !mbar_wait_bounded(&empty[st], (k - 1) & 1, pool.status)) break;
       const int j = j0 + i;
-      const int tier = p.tier_map[rowbase + j];
-      const int64_t phys = p.table[rowbase + j];
+      const int tier = __shfl_sync(0xffffffffu, pf_tier, i & 31);
+      const int64_t phys = __shfl_sync(0xffffffffu, pf_phys, i & 31);
       const int ntok = min(kT, ctx - j * kT);
       bool valid = true;
       if (tier > 1) {
@@ -139,7 +182,7 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ?
       }
       const uint16_t* kp = tier_base(pool, tier) + chunk_offset(pool, tier, p.layer, phys, 0, g);
       const uint16_t* vp = tier_base(pool, tier) + chunk_offset(pool, tier, p.layer, phys, 1, g);
-      if (tier == DKV_TIER_HBM) {
+      if (tier == DKV_TIER_HBM && !p.lsu_hbm) {
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
           mbar_arrive(&full[st]);
@@ -170,7 +213,8 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ?
   const int tg = lane >> 3, dg = lane & 7;
   const int hbase = g * C::G + hq * HPW;  // first global q head of this warp
 
-  float qreg[HPW][C::QCH][8];
+  // q of this lane's key dims, as (even, odd) dim pairs for the packed fp32x2 FMA
+  float2 q2[HPW][C::QCH][4];
 #pragma unroll
   for (int h = 0; h < HPW; ++h)
 #pragma unroll
@@ -178,19 +222,22 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ?
       const float4* src = reinterpret_cast<const float4*>(
           p.qs + ((int64_t)b * p.Hq + hbase + h) * D + (dg + 8 * hh) * 8);
       const float4 a = src[0], c = src[1];
-      qreg[h][hh][0] = a.x; qreg[h][hh][1] = a.y; qreg[h][hh][2] = a.z; qreg[h][hh][3] = a.w;
-      qreg[h][hh][4] = c.x; qreg[h][hh][5] = c.y; qreg[h][hh][6] = c.z; qreg[h][hh][7] = c.w;
+      q2[h][hh][0] = make_float2(a.x, a.y);
+      q2[h][hh][1] = make_float2(a.z, a.w);
+      q2[h][hh][2] = make_float2(c.x, c.y);
+      q2[h][hh][3] = make_float2(c.z, c.w);
     }
 
-  float acc[HPW][C::DPL];
+  constexpr int NP = C::DPL / 2;  // value-dim pairs per lane
+  float2 acc2[HPW][NP];
 #pragma unroll
   for (int h = 0; h < HPW; ++h)
 #pragma unroll
-    for (int e = 0; e < C::DPL; ++e) acc[h][e] = 0.f;
+    for (int e = 0; e < NP; ++e) acc2[h][e] = make_float2(0.f, 0.f);
   float m_run = -INFINITY, l_run = 0.f;  // state of head h_lane (lane-group uniform m)
   const int h_lane = dg >> (3 - C::LOGH);
   const bool head_leader = tg == 0 && (dg & C::LOWMASK) == 0;
-  float* pb = pbuf + warp * kT * HPW;
+  float2* pb = pbuf + warp * kT * HPW;   // (p, p) per (token, head)
   float* al = alph + warp * HPW;
 
   for (int i = slot; i < n_local; i += kSlots) {
@@ -201,24 +248,35 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ?
       const uint16_t* Ks = stages + st * C::STAGE_ELEMS;
       const uint16_t* Vs = Ks + kT * D;
       // ---- partial scores: lane (tg, dg) covers tokens tg + 4 i4 and 16-byte key
-      // chunks dg + 8 hh (eight lanes read one 128-byte row segment: no bank conflicts)
-      float v[C::NV];
+      // chunks dg + 8 hh (eight lanes read one 128-byte row segment: no bank conflicts);
+      // even and odd dims accumulate in the two halves of a packed pair
+      float2 v2[C::NV];
 #pragma unroll
-      for (int x = 0; x < C::NV; ++x) v[x] = 0.f;
+      for (int x = 0; x < C::NV; ++x) v2[x] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int i4 = 0; i4 < 4; ++i4) {
         const int t = tg + 4 * i4;
 #pragma unroll
         for (int hh = 0; hh < C::QCH; ++hh) {
           const uint4 w = *reinterpret_cast<const uint4*>(Ks + t * D + (dg + 8 * hh) * 8);
-          const float kf[8] = {bf16lo(w.x), bf16hi(w.x), bf16lo(w.y), bf16hi(w.y),
-                               bf16lo(w.z), bf16hi(w.z), bf16lo(w.w), bf16hi(w.w)};
+          const float2 k0 = make_float2(bf16lo(w.x), bf16hi(w.x));
+          const float2 k1 = make_float2(bf16lo(w.y), bf16hi(w.y));
+          const float2 k2 = make_float2(bf16lo(w.z), bf16hi(w.z));
+          const float2 k3 = make_float2(bf16lo(w.w), bf16hi(w.w));
 #pragma unroll
-          for (int h = 0; h < HPW; ++h)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[h * 4 + i4] = fmaf(qreg[h][hh][e], kf[e], v[h * 4 + i4]);
+          for (int h = 0; h < HPW; ++h) {
+            float2 a = v2[h * 4 + i4];
+            a = __ffma2_rn(q2[h][hh][0], k0, a);
+            a = __ffma2_rn(q2[h][hh][1], k1, a);
+            a = __ffma2_rn(q2[h][hh][2], k2, a);
+            a = __ffma2_rn(q2[h][hh][3], k3, a);
+            v2[h * 4 + i4] = a;
+          }
         }
       }
+      float v[C::NV];
+#pragma unroll
+      for (int x = 0; x < C::NV; ++x) v[x] = v2[x].x + v2[x].y;
       // ---- reduce-scatter over the 8 dg lanes (masks 4, 2, 1): value index h*4+i4
       rs_level<C::NV>(v, (dg & 4) != 0, 4);
       rs_level<(C::NV >= 2 ? C::NV / 2 : 1)>(v, (dg & 2) != 0, 2);
@@ -247,7 +305,7 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ?
       for (int r = 0; r < C::NR; ++r) {
         const float pr = fast_exp2(sv[r] - m_use);
         if (C::NV >= 8 || (dg & 1) == 0) {
-          pb[tk[r] * HPW + h_lane] = pr;
+          pb[tk[r] * HPW + h_lane] = make_float2(pr, pr);
           psum += pr;
         }
       }
@@ -255,38 +313,42 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ?
       m_run = m_new;
       if (head_leader) al[h_lane] = alpha;
       __syncwarp();
-      // ---- P.V: lane owns value dims [lane*DPL, lane*DPL + DPL)
-      float a_h[HPW];
+      // ---- P.V: lane owns value dims [lane*DPL, lane*DPL + DPL) as packed pairs
 #pragma unroll
-      for (int h = 0; h < HPW; ++h) a_h[h] = al[h];
+      for (int h = 0; h < HPW; ++h) {
+        const float a = al[h];
+        const float2 a2 = make_float2(a, a);
 #pragma unroll
-      for (int h = 0; h < HPW; ++h)
-#pragma unroll
-        for (int e = 0; e < C::DPL; ++e) acc[h][e] *= a_h[h];
+        for (int e = 0; e < NP; ++e) acc2[h][e] = __fmul2_rn(acc2[h][e], a2);
+      }
       const int d0 = lane * C::DPL;
 #pragma unroll
       for (int t = 0; t < kT; ++t) {
         if (t < ntok) {
-          float vf[C::DPL];
-          if constexpr (C::DPL == 4) {
+          float2 vf[NP];
+          if constexpr (NP == 2) {
             const uint2 w = *reinterpret_cast<const uint2*>(Vs + t * D + d0);
-            vf[0] = bf16lo(w.x); vf[1] = bf16hi(w.x); vf[2] = bf16lo(w.y); vf[3] = bf16hi(w.y);
+            vf[0] = make_float2(bf16lo(w.x), bf16hi(w.x));
+            vf[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
           } else {
             const uint32_t w = *reinterpret_cast<const uint32_t*>(Vs + t * D + d0);
-            vf[0] = bf16lo(w); vf[1] = bf16hi(w);
+            vf[0] = make_float2(bf16lo(w), bf16hi(w));
           }
-          float pp[HPW];
-          if constexpr (HPW == 4) {
-            const float4 q4 = *reinterpret_cast<const float4*>(pb + t * 4);
-            pp[0] = q4.x; pp[1] = q4.y; pp[2] = q4.z; pp[3] = q4.w;
-          } else {
+          float2 pp[HPW];
+          if constexpr (HPW >= 2) {
 #pragma unroll
-            for (int h = 0; h < HPW; ++h) pp[h] = pb[t * HPW + h];
+            for (int h2 = 0; h2 < HPW; h2 += 2) {
+              const float4 q4 = *reinterpret_cast<const float4*>(pb + t * HPW + h2);
+              pp[h2] = make_float2(q4.x, q4.y);
+              pp[h2 + 1] = make_float2(q4.z, q4.w);
+            }
+          } else {
+            pp[0] = pb[t];
           }
 #pragma unroll
           for (int h = 0; h < HPW; ++h)
 #pragma unroll
-            for (int e = 0; e < C::DPL; ++e) acc[h][e] = fmaf(pp[h], vf[e], acc[h][e]);
+            for (int e = 0; e < NP; ++e) acc2[h][e] = __ffma2_rn(pp[h], vf[e], acc2[h][e]);
         }
       }
     }
@@ -307,7 +369,8 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ?
 #pragma unroll
   for (int h = 0; h < HPW; ++h)
 #pragma unroll
-    for (int e = 0; e < C::DPL; ++e) macc[(warp * HPW + h) * D + lane * C::DPL + e] = acc[h][e];
+    for (int e = 0; e < NP; ++e)
+      *reinterpret_cast<float2*>(macc + (warp * HPW + h) * D + lane * C::DPL + 2 * e) = acc2[h][e];
   if (head_leader) mml[warp * HPW + h_lane] = make_float2(m_run, l_tot);
   named_bar_sync(1, C::NCW * 32);
 
@@ -331,6 +394,34 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, WPB == 1 ?
     p.part_acc[base * D + d] = A;
     if (d == 0) p.part_ml[base] = make_float2(M, Ls);
   }
+
+  // ---- fused combine: the last split CTA of (b, g) to finish merges all S partial states
+  // (in split order, so the result does not depend on which CTA finishes last)
+  if (p.out) {
+    __shared__ int s_last;
+    __shared__ float s_new[8];
+    __threadfence();
+    named_bar_sync(1, C::NCW * 32);
+    if (threadIdx.x == 0) s_last = atomicAdd(p.cnt + (int64_t)b * pool.Hkv + g, 1) == p.S - 1;
+    named_bar_sync(1, C::NCW * 32);
+    if (s_last) {
+      __threadfence();
+      const float* kn = p.knew + ((int64_t)b * pool.Hkv + g) * D;
+      for (int hh = warp; hh < C::G; hh += C::NCW) {
+        const float sc = new_token_score(p.qs + ((int64_t)b * p.Hq + g * C::G + hh) * D, kn, D, lane);
+        if (lane == 0) s_new[hh] = sc;
+      }
+      named_bar_sync(1, C::NCW * 32);
+      for (int o = threadIdx.x; o < C::G * D; o += C::NCW * 32) {
+        const int hh = o / D, d = o % D;
+        const int hg = g * C::G + hh;
+        const float r = combine_value(p.part_ml, p.part_acc, p.S, ((int64_t)b * p.Hq + hg) * p.S, D, d,
+                                      s_new[hh], p.vnew[((int64_t)b * pool.Hkv + g) * D + d]);
+        p.out[((int64_t)b * p.Hq + hg) * D + d] = f32_to_bf16_bits(r);
+      }
+      if (threadIdx.x == 0) p.cnt[(int64_t)b * pool.Hkv + g] = 0;
+    }
+  }
 }
 
 // ----------------------------------------------------------------------- combine
@@ -341,36 +432,29 @@ template <int D>
 __global__ void __launch_bounds__(D) combine_kernel(int Hq, int Hkv, int S,
                                                     const float2* __restrict__ ml,
                                                     const float* __restrict__ acc,
-                                                    const float* __restrict__ snew,
+                                                    const float* __restrict__ qs,
+                                                    const float* __restrict__ knew,
                                                     const float* __restrict__ vnew,
                                                     uint16_t* __restrict__ out) {
   const int hg = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
   const int g = hg / (Hq / Hkv);
-  const int64_t base = ((int64_t)b * Hq + hg) * S;
-  const float sn = snew[(int64_t)b * Hq + hg];
-  float M = sn;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, ml[base + s].x);
-  const float wn = exp2f(sn - M);
-  float L = wn;
-  float A = wn * vnew[((int64_t)b * Hkv + g) * D + d];
-  for (int s = 0; s < S; ++s) {
-    const float2 m = ml[base + s];
-    if (m.x != -INFINITY) {
-      const float w = exp2f(m.x - M);
-      L = fmaf(m.y, w, L);
-      A = fmaf(acc[(base + s) * D + d], w, A);
-    }
+  __shared__ float s_new;
+  if (d < 32) {
+    const float sc = new_token_score(qs + ((int64_t)b * Hq + hg) * D, knew + ((int64_t)b * Hkv + g) * D, D, d);
+    if (d == 0) s_new = sc;
   }
-  out[((int64_t)b * Hq + hg) * D + d] = f32_to_bf16_bits(A / L);
+  __syncthreads();
+  const float r = combine_value(ml, acc, S, ((int64_t)b * Hq + hg) * S, D, d, s_new,
+                                vnew[((int64_t)b * Hkv + g) * D + d]);
+  out[((int64_t)b * Hq + hg) * D + d] = f32_to_bf16_bits(r);
 }
 
 // ---------------------------------------------------------------------- launchers
 
-template <int D, int HPW, int WPB>
+template <int D, int HPW, int WPB, int NST, int MINB>
 static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
-  constexpr int NST = 8;
   using C = AttnCfg<D, HPW, WPB, NST>;
-  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST>;
+  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB>;
   static bool attr_done = false;  // per instantiation
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -382,32 +466,38 @@ static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
   return cuda_check(cudaGetLastError(), "attention launch");
 }
 
-int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, cudaStream_t st) {
-  if (D == 128) {
-    switch (G) {
-      case 1: return launch_attn_t<128, 1, 1>(p, B, Hkv, st);
-      case 2: return launch_attn_t<128, 2, 1>(p, B, Hkv, st);
-      case 4: return launch_attn_t<128, 4, 1>(p, B, Hkv, st);
-      case 8: return launch_attn_t<128, 4, 2>(p, B, Hkv, st);
-    }
-  } else if (D == 64) {
-    switch (G) {
-      case 1: return launch_attn_t<64, 1, 1>(p, B, Hkv, st);
-      case 2: return launch_attn_t<64, 2, 1>(p, B, Hkv, st);
-      case 4: return launch_attn_t<64, 4, 1>(p, B, Hkv, st);
-      case 8: return launch_attn_t<64, 4, 2>(p, B, Hkv, st);
-    }
+// Kernel shape per (D, G) and variant: 0 = default; 1 = 12-stage ring; 2 = two warps per
+// block with G/2 heads each (G = 4); 3 = both.
+template <int D>
+static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_attn_t<D, 1, 1, 8, 3>(p, B, Hkv, st);
+    case 2: return launch_attn_t<D, 2, 1, 8, 3>(p, B, Hkv, st);
+    case 4:
+      switch (variant) {
+        case 1: return launch_attn_t<D, 4, 1, 12, 2>(p, B, Hkv, st);
+        case 2: return launch_attn_t<D, 2, 2, 8, 2>(p, B, Hkv, st);
+        case 3: return launch_attn_t<D, 2, 2, 12, 2>(p, B, Hkv, st);
+        default: return launch_attn_t<D, 4, 1, 8, 3>(p, B, Hkv, st);
+      }
+    case 8: return launch_attn_t<D, 4, 2, 8, 1>(p, B, Hkv, st);
   }
-  return set_error(DKV_ERR_UNSUPPORTED, "attention: unsupported D=%d G=%d", D, G);
+  return set_error(DKV_ERR_UNSUPPORTED, "attention: unsupported G=%d", G);
+}
+
+int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, int variant, cudaStream_t st) {
+  if (D == 128) return launch_attn_d<128>(p, B, Hkv, G, variant, st);
+  if (D == 64) return launch_attn_d<64>(p, B, Hkv, G, variant, st);
+  return set_error(DKV_ERR_UNSUPPORTED, "attention: unsupported D=%d", D);
 }
 
 int launch_combine(int B, int Hq, int Hkv, int D, int S, const float2* ml, const float* acc,
-                   const float* snew, const float* vnew, uint16_t* out, cudaStream_t st) {
+                   const float* qs, const float* knew, const float* vnew, uint16_t* out, cudaStream_t st) {
   dim3 grid(Hq, B);
   if (D == 128)
-    combine_kernel<128><<<grid, 128, 0, st>>>(Hq, Hkv, S, ml, acc, snew, vnew, out);
+    combine_kernel<128><<<grid, 128, 0, st>>>(Hq, Hkv, S, ml, acc, qs, knew, vnew, out);
   else
-    combine_kernel<64><<<grid, 64, 0, st>>>(Hq, Hkv, S, ml, acc, snew, vnew, out);
+    combine_kernel<64><<<grid, 64, 0, st>>>(Hq, Hkv, S, ml, acc, qs, knew, vnew, out);
   return cuda_check(cudaGetLastError(), "combine launch");
 }
 

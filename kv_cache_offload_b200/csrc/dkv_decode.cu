@@ -3,11 +3,10 @@
 //
 // DirectKV ("长上下文 LLM 的零拷贝 KV Cache 卸载（OSDI 2026）", 核心方法) fuses KV generation
 // (the QKV projection) with attention so that the new K/V are consumed on chip and never
-// written out and read back. Here the projection's epilogue owns one kv-head group
-// (its G query heads plus the group's key and value rows), so it has everything the new
-// token's attention term needs: it rotates q and k, writes bf16 k_hat/v_hat to the cache
-// exactly once, and emits the new token's softmax partial (score q.k_hat, value v_hat),
-// which the combine stage folds in. The attention stage then reads only cached blocks.
+// written out and read back. Here the projection's epilogue rotates q and k, writes bf16
+// k_hat / v_hat to the cache exactly once, and leaves q, k_hat, v_hat (fp32) in the
+// workspace; the attention stage reads only the cached blocks, and its combine folds in
+// the new token's term (score q . k_hat, value v_hat) without re-reading the cache.
 #include <math.h>
 
 #include "dkv_internal.h"
@@ -43,8 +42,9 @@ int decode_ws_layout(const dkv_pool* pool, int B, int max_blocks, int Hq, int hi
   w->S = pick_attn_splits(pool, B, Hkv, max_blocks);
   size_t o = 0;
   w->off_qs = o;       o = align_up(o + (size_t)B * Hq * D * 4, 256);
-  w->off_snew = o;     o = align_up(o + (size_t)B * Hq * 4, 256);
+  w->off_knew = o;     o = align_up(o + (size_t)B * Hkv * D * 4, 256);
   w->off_vnew = o;     o = align_up(o + (size_t)B * Hkv * D * 4, 256);
+  w->off_cnt = o;      o = align_up(o + (size_t)B * Hkv * 4, 256);
   w->off_ml = o;       o = align_up(o + (size_t)B * Hq * w->S * 8, 256);
   w->off_acc = o;      o = align_up(o + (size_t)B * Hq * w->S * D * 4, 256);
   w->total = o;
@@ -107,15 +107,16 @@ int dkv_decode_project(dkv_pool* pool, int layer, const uint16_t* x, const uint1
   a.theta = (double)rope_theta;
   a.qscale = (float)(1.4426950408889634 / sqrt((double)w.D));
   a.qs = reinterpret_cast<float*>(ws + w.off_qs);
-  a.snew = reinterpret_cast<float*>(ws + w.off_snew);
+  a.knew = reinterpret_cast<float*>(ws + w.off_knew);
   a.vnew = reinterpret_cast<float*>(ws + w.off_vnew);
+  a.attn_cnt = reinterpret_cast<int*>(ws + w.off_cnt);
   a.cluster = pool->tuning.proj_splits;
   return launch_projection(a, (cudaStream_t)stream);
 }
 
 int dkv_decode_attend(dkv_pool* pool, int layer, const int32_t* block_table, const int32_t* seq_lens,
                       const uint8_t* tier_map, int B, int max_blocks, int hidden, int num_q_heads,
-                      void* workspace, size_t ws_bytes, void* stream) {
+                      uint16_t* out, void* workspace, size_t ws_bytes, void* stream) {
   if (!pool || !block_table || !seq_lens || !tier_map)
     return set_error(DKV_ERR_ARG, "dkv_decode_attend: null argument");
   DecodeWs w;
@@ -135,7 +136,12 @@ int dkv_decode_attend(dkv_pool* pool, int layer, const int32_t* block_table, con
   a.qs = reinterpret_cast<const float*>(ws + w.off_qs);
   a.part_ml = reinterpret_cast<float2*>(ws + w.off_ml);
   a.part_acc = reinterpret_cast<float*>(ws + w.off_acc);
-  return launch_attention(a, B, w.Hkv, w.D, w.G, (cudaStream_t)stream);
+  a.cnt = reinterpret_cast<int*>(ws + w.off_cnt);
+  a.knew = reinterpret_cast<const float*>(ws + w.off_knew);
+  a.vnew = reinterpret_cast<const float*>(ws + w.off_vnew);
+  a.out = out;
+  a.lsu_hbm = pool->tuning.attn_lsu_hbm;
+  return launch_attention(a, B, w.Hkv, w.D, w.G, pool->tuning.attn_variant, (cudaStream_t)stream);
 }
 
 int dkv_decode_combine(dkv_pool* pool, int B, int max_blocks, int hidden, int num_q_heads, uint16_t* out,
@@ -147,8 +153,9 @@ int dkv_decode_combine(dkv_pool* pool, int B, int max_blocks, int hidden, int nu
   if ((rc = check_common(pool, 0, workspace, ws_bytes, w))) return rc;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   return launch_combine(B, num_q_heads, w.Hkv, w.D, w.S, reinterpret_cast<const float2*>(ws + w.off_ml),
-                        reinterpret_cast<const float*>(ws + w.off_acc), reinterpret_cast<const float*>(ws + w.off_snew),
-                        reinterpret_cast<const float*>(ws + w.off_vnew), out, (cudaStream_t)stream);
+                        reinterpret_cast<const float*>(ws + w.off_acc), reinterpret_cast<const float*>(ws + w.off_qs),
+                        reinterpret_cast<const float*>(ws + w.off_knew), reinterpret_cast<const float*>(ws + w.off_vnew),
+                        out, (cudaStream_t)stream);
 }
 
 int dkv_decode_step(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t* Wqkv, const int32_t* block_table,
@@ -159,10 +166,8 @@ int dkv_decode_step(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t
   int rc = dkv_decode_project(pool, layer, x, Wqkv, block_table, seq_lens, tier_map, B, max_blocks, hidden,
                               num_q_heads, rope_theta, workspace, ws_bytes, stream);
   if (rc) return rc;
-  rc = dkv_decode_attend(pool, layer, block_table, seq_lens, tier_map, B, max_blocks, hidden, num_q_heads,
-                         workspace, ws_bytes, stream);
-  if (rc) return rc;
-  return dkv_decode_combine(pool, B, max_blocks, hidden, num_q_heads, out, workspace, ws_bytes, stream);
+  return dkv_decode_attend(pool, layer, block_table, seq_lens, tier_map, B, max_blocks, hidden, num_q_heads,
+                           out, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"

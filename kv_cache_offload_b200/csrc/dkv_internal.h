@@ -58,11 +58,17 @@ struct AttnParams {
   const float* qs;   // [B][Hq][D], scaled by log2(e)/sqrt(D)
   float2* part_ml;   // [B][Hq][S] (m, l)
   float* part_acc;   // [B][Hq][S][D]
+  // fused combine (when out != nullptr): the last CTA of each (b, kv head) merges
+  int* cnt;          // [B][Hkv] arrival counters (zero on entry)
+  const float* knew; // [B][Hkv][D]
+  const float* vnew; // [B][Hkv][D]
+  uint16_t* out;     // [B][Hq*D] bf16, or nullptr
+  int lsu_hbm;       // load HBM-tier blocks with cp.async instead of bulk copies
 };
 
-int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, cudaStream_t st);
+int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, int variant, cudaStream_t st);
 int launch_combine(int B, int Hq, int Hkv, int D, int S, const float2* ml, const float* acc,
-                   const float* snew, const float* vnew, uint16_t* out, cudaStream_t st);
+                   const float* qs, const float* knew, const float* vnew, uint16_t* out, cudaStream_t st);
 
 // Arguments of one projection launch (see dkv_projection.cu).
 struct ProjArgs {
@@ -78,8 +84,9 @@ struct ProjArgs {
   double theta;
   float qscale;   // log2(e) / sqrt(D)
   float* qs;      // [B][Hq][D]
-  float* snew;    // [B][Hq]
-  float* vnew;    // [B][Hkv][D]
+  float* knew;    // [B][Hkv][D]  k_hat as fp32
+  float* vnew;    // [B][Hkv][D]  v_hat as fp32
+  int* attn_cnt;  // [B][Hkv] attention split counters, reset by the projection
   int cluster;    // cluster size request (0 = automatic)
 };
 
@@ -88,7 +95,7 @@ int launch_projection(const ProjArgs& a, cudaStream_t st);
 // Workspace carve-up of one decode step (all offsets 256-byte aligned).
 struct DecodeWs {
   int B, Hq, Hkv, D, rows, S, G, max_blocks, hidden;
-  size_t off_qs, off_snew, off_vnew, off_ml, off_acc, total;
+  size_t off_qs, off_knew, off_vnew, off_cnt, off_ml, off_acc, total;
 };
 
 // Fills `w` for a shape; returns DKV_OK or an error (unsupported shape).

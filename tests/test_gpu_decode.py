@@ -180,3 +180,23 @@ def test_layout_conversion_bit_exact(src_tier):
             assert np.array_equal(back.cpu().view(torch.int16).numpy().view(np.uint16), bits.reshape(-1))
         finally:
             ctx.close()
+
+
+def test_staged_calls_match_fused_step():
+    # project; attend(out=None); combine  ==  project; attend(out)  ==  dkv_decode_step
+    cfg = WL.small_config(B=4, ctx_range=(100, 400), host_prob=0.4)
+    inp = WL.make_decode_inputs(cfg, seed=5)
+    ctx = TL.make_pool(inp)
+    try:
+        fused = TL.run_step(ctx, layer=1)
+        x, W = inp.x.cuda(), inp.W.cuda()
+        nws = dkv.dkv_decode_workspace_bytes(ctx.pool, cfg.B, ctx.table.shape[1], cfg.Hq, cfg.H)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        staged = torch.empty_like(fused)
+        dkv.dkv_decode_project(ctx.pool, 1, x, W, ctx.table, ctx.seq_lens, ctx.tier_map, cfg.Hq, cfg.theta, ws)
+        dkv.dkv_decode_attend(ctx.pool, 1, ctx.table, ctx.seq_lens, ctx.tier_map, cfg.H, cfg.Hq, ws)
+        dkv.dkv_decode_combine(ctx.pool, cfg.B, ctx.table.shape[1], cfg.H, cfg.Hq, staged, ws)
+        assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
+        assert torch.equal(staged, fused)
+    finally:
+        ctx.close()
