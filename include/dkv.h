@@ -220,6 +220,43 @@ int dkv_permute_layout(const void* src, void* dst, int src_layout, int num_layer
 int dkv_convert_layout(dkv_pool* pool, int tier, void* dst, size_t dst_bytes, void* stream);
 
 /*
+ * Zero-copy GEMM study (DirectKV's motivating experiment, Fig. 2(a) as quoted in
+ * "「KV Cache 内存层级」系列总纲", §一 and §四; CPU-aware tiling, §2.1):
+ *   C[M][N] (fp32) = A[M][K] (bf16, device memory) . B[K][N], with B stored column-major as
+ *   Bt[N][K] (bf16; Bt[n][k] = B[k][n]) in mapped pinned host memory (pass its device
+ *   alias) or, for DKV_GEMM_DEVICE, in device memory.
+ * Variants:
+ *   DKV_GEMM_CPU_AWARE        B-panel-major tile order: each B tile crosses the host link
+ *                             once and is reused from L2; A is re-read from HBM per panel.
+ *   DKV_GEMM_NAIVE_ZERO_COPY  row-major tile order: B re-read over the host link by every
+ *                             128-row tile row of C.
+ *   DKV_GEMM_STAGED_SWAP      cudaMemcpyAsync of all of B into the workspace ("swap" into a
+ *                             GPU buffer), then the product from device memory.
+ *   DKV_GEMM_DEVICE           A and Bt both in device memory.
+ * Shapes: M % 128 == 0, N % 256 == 0, K % 64 == 0 (else DKV_ERR_UNSUPPORTED). Pointers
+ * 256-byte aligned. workspace >= dkv_gemm_workspace_bytes(variant, M, N, K): its first 4
+ * bytes are a device status word the kernel clears and sets on a device-side timeout;
+ * DKV_GEMM_STAGED_SWAP also holds the staged copy of B there. fp32 accumulation on the
+ * tensor cores (tcgen05, bf16 inputs).
+ */
+/*
+ * Mapped pinned host memory for operands read zero-copy (e.g. B of the GEMM study):
+ * cudaHostAlloc(mapped [| write-combined]); `dev_ptr` receives the device alias.
+ * Free with dkv_host_free. Errors: DKV_ERR_ARG, DKV_ERR_OOM.
+ */
+int dkv_host_alloc_mapped(size_t bytes, int host_flags, void** host_ptr, void** dev_ptr);
+int dkv_host_free(void* host_ptr);
+
+#define DKV_GEMM_CPU_AWARE       0
+#define DKV_GEMM_NAIVE_ZERO_COPY 1
+#define DKV_GEMM_STAGED_SWAP     2
+#define DKV_GEMM_DEVICE          3
+
+size_t dkv_gemm_workspace_bytes(int variant, int M, int N, int K);
+int dkv_gemm(int variant, const uint16_t* A, const uint16_t* Bt, float* C, int M, int N, int K,
+             void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Synchronise `stream`, then read and clear the pool's device status word.
  * Returns DKV_OK, DKV_ERR_BAD_TABLE (a kernel skipped a block with a bad tier or physical
  * id, or a context exceeding max_blocks*T), DKV_ERR_TIMEOUT, or DKV_ERR_CUDA.

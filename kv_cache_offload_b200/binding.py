@@ -30,6 +30,10 @@ DKV_TIER_HOST = 1
 DKV_LAYOUT_LAYER_FIRST = 0
 DKV_LAYOUT_PAGE_FIRST = 1
 DKV_HOST_WRITE_COMBINED = 1
+DKV_GEMM_CPU_AWARE = 0
+DKV_GEMM_NAIVE_ZERO_COPY = 1
+DKV_GEMM_STAGED_SWAP = 2
+DKV_GEMM_DEVICE = 3
 
 
 class DkvError(RuntimeError):
@@ -75,6 +79,10 @@ _SIGS = {
     "dkv_permute_layout": (_I, [_P, _P, _I, _I, _I64, _I64, _P]),
     "dkv_convert_layout": (_I, [_P, _I, _P, _SZ, _P]),
     "dkv_check": (_I, [_P, _P]),
+    "dkv_gemm_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
+    "dkv_host_alloc_mapped": (_I, [_SZ, _I, ctypes.POINTER(_P), ctypes.POINTER(_P)]),
+    "dkv_host_free": (_I, [_P]),
+    "dkv_gemm": (_I, [_I, _P, _P, _P, _I, _I, _I, _P, _SZ, _P]),
     "dkv_last_error": (ctypes.c_char_p, []),
     "dkv_version": (ctypes.c_char_p, []),
 }
@@ -290,6 +298,51 @@ def dkv_convert_layout(pool: int, tier: int, dst, dst_bytes: Optional[int] = Non
     if dst_bytes is None:
         dst_bytes = dst.numel() * dst.element_size()
     _chk(lib().dkv_convert_layout(pool, tier, _ptr(dst), dst_bytes, _stream(stream)))
+
+
+class MappedHostBuffer:
+    """Mapped pinned host memory from dkv_host_alloc_mapped: `.tensor` is a CPU view of
+    `numel` elements of `dtype`, `.dev_ptr` the device alias. Freed by close()."""
+
+    def __init__(self, numel: int, dtype=torch.int16, host_flags: int = 0):
+        import numpy as np
+        esz = torch.empty(0, dtype=dtype).element_size()
+        h, d = _P(), _P()
+        _chk(lib().dkv_host_alloc_mapped(numel * esz, host_flags, ctypes.byref(h), ctypes.byref(d)))
+        self.host_ptr, self.dev_ptr, self.numel = h.value, d.value, numel
+        raw = (ctypes.c_uint8 * (numel * esz)).from_address(self.host_ptr)
+        self.tensor = torch.from_numpy(np.ctypeslib.as_array(raw)).view(dtype)
+
+    def close(self):
+        if self.host_ptr:
+            self.tensor = None
+            _chk(lib().dkv_host_free(self.host_ptr))
+            self.host_ptr = 0
+
+
+def dkv_host_alloc_mapped(numel: int, dtype=torch.int16, host_flags: int = 0) -> "MappedHostBuffer":
+    return MappedHostBuffer(numel, dtype, host_flags)
+
+
+def dkv_host_free(buf: "MappedHostBuffer"):
+    buf.close()
+
+
+def dkv_gemm_workspace_bytes(variant: int, M: int, N: int, K: int) -> int:
+    return lib().dkv_gemm_workspace_bytes(variant, M, N, K)
+
+
+def dkv_gemm(variant: int, A: torch.Tensor, Bt, C: torch.Tensor, workspace: torch.Tensor, M: int = 0,
+             N: int = 0, K: int = 0, stream=None):
+    """C = A . B with Bt = B^T ([N][K]); Bt may be a device tensor or a raw device pointer
+    (e.g. the device alias of mapped pinned host memory), then give M, N, K explicitly."""
+    _need(A, torch.bfloat16, "A")
+    _need(C, torch.float32, "C")
+    M = M or A.shape[0]
+    K = K or A.shape[1]
+    N = N or C.shape[1]
+    _chk(lib().dkv_gemm(variant, _ptr(A), _ptr(Bt), _ptr(C), M, N, K, _ptr(workspace),
+                        workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def dkv_check(pool: int, stream=None) -> int:

@@ -282,6 +282,33 @@ int dkv_convert_layout(dkv_pool* p, int tier, void* dst, size_t dst_bytes, void*
   return dkv_permute_layout(src, dst, p->cfg.layout, p->cfg.num_layers, blocks, chunk, stream);
 }
 
+int dkv_host_alloc_mapped(size_t bytes, int host_flags, void** host_ptr, void** dev_ptr) {
+  if (!host_ptr || !dev_ptr || bytes == 0 || (host_flags & ~DKV_HOST_WRITE_COMBINED))
+    return set_error(DKV_ERR_ARG, "dkv_host_alloc_mapped: bad argument");
+  unsigned flags = cudaHostAllocMapped | cudaHostAllocPortable;
+  if (host_flags & DKV_HOST_WRITE_COMBINED) flags |= cudaHostAllocWriteCombined;
+  void* h = nullptr;
+  cudaError_t e = cudaHostAlloc(&h, bytes, flags);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return set_error(DKV_ERR_OOM, "dkv_host_alloc_mapped: %zu bytes: %s", bytes, cudaGetErrorString(e));
+  }
+  void* d = nullptr;
+  e = cudaHostGetDevicePointer(&d, h, 0);
+  if (e != cudaSuccess) {
+    cudaFreeHost(h);
+    return cuda_check(e, "dkv_host_alloc_mapped: cudaHostGetDevicePointer");
+  }
+  *host_ptr = h;
+  *dev_ptr = d;
+  return DKV_OK;
+}
+
+int dkv_host_free(void* host_ptr) {
+  if (!host_ptr) return set_error(DKV_ERR_ARG, "dkv_host_free: null pointer");
+  return cuda_check(cudaFreeHost(host_ptr), "dkv_host_free");
+}
+
 int dkv_check(dkv_pool* p, void* stream) {
   if (!p) return set_error(DKV_ERR_ARG, "dkv_check: null pool");
   int rc = cuda_check(cudaStreamSynchronize((cudaStream_t)stream), "dkv_check: stream sync");
