@@ -46,6 +46,7 @@ def parse():
     ap.add_argument("--host-flags", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
+    ap.add_argument("--gemm-dim", type=int, default=0, help="override M=N=K of the GEMM study (profiling)")
     ap.add_argument("--profile", action="store_true",
                     help="warm-up + timed steps only (no clock pre-roll, e2e or CPU baseline): for ncu")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
@@ -340,6 +341,8 @@ def run_gemm(args, rank, world):
     dev = torch.device("cuda", local)
     cfg = WL.GEMM_CONFIGS["gemm"]
     M, N, K = cfg.M, cfg.N, cfg.K
+    if args.gemm_dim:
+        M = N = K = args.gemm_dim
     gen = torch.Generator(device=dev)
     gen.manual_seed(rank)
     A = (torch.rand((M, K), generator=gen, device=dev) * 2 - 1).to(torch.bfloat16)
@@ -373,8 +376,8 @@ def run_gemm(args, rank, world):
     line = {"metric": "zero-copy GEMM 10240^3 time (CPU-aware tiling)", "value": ca, "unit": "ms",
             "higher_is_better": False, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "dtype": "bf16", "data": "synthetic", "impl": "dkv",
-            "config": {"workload": "gemm: C = A.B, M=N=K=10240, A bf16 in HBM, B bf16 column-major in mapped "
-                                   "pinned host memory, fp32 accumulate/output"},
+            "config": {"workload": "gemm: C = A.B, M=N=K=%d, A bf16 in HBM, B bf16 column-major in mapped "
+                                   "pinned host memory, fp32 accumulate/output" % M},
             "variants": res,
             "host_link": {"h2d_peak_gbs": h2d, "algorithmic_host_bytes": b_bytes,
                           "cpu_aware_link_gbs": b_bytes / (ca * 1e-3) / 1e9,
