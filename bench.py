@@ -40,7 +40,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="dkv", choices=["dkv", "reference"])
-    ap.add_argument("--config", default="8b_hbm", choices=sorted(WL.CONFIGS) + ["gemm"])
+    ap.add_argument("--config", default="8b_hbm", choices=sorted(WL.CONFIGS) + ["gemm", "layout"])
+    ap.add_argument("--compare-staged", action="store_true",
+                    help="host-tier configs: also time swap-in (DMA and copy kernel) + HBM attention")
     ap.add_argument("--attn-splits", type=int, default=0)
     ap.add_argument("--proj-splits", type=int, default=0)
     ap.add_argument("--host-flags", type=int, default=0)
@@ -138,6 +140,22 @@ class ClockSampler:
         sm.sort()
         return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+def reduce_max_over_ranks(vals, dist: bool, device=None):
+    """Element-wise max over ranks of per-rank timings (ms); identity without a process
+    group. Every rank calls it the same number of times (it is a collective)."""
+    t = torch.tensor(list(vals), dtype=torch.float64, device=device)
+    if dist:
+        import torch.distributed as tdist
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def replica_throughput(tokens_per_rank: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas: all ranks' tokens over the
+    slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step_max * 1e-3)
 
 
 # ------------------------------------------------------------------ GPU workload
@@ -388,8 +406,110 @@ def run_gemm(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def run_layout(args):
+    """Block-layout permutation (layer-first -> page-first) of a 2 GiB tier: L=32 layers,
+    1024 blocks, 8 kv heads, D=128, T=16; HBM -> HBM and mapped host -> HBM."""
+    import kv_cache_offload_b200 as dkv
+    from kv_cache_offload_b200.build import build
+    build()
+    dev = torch.device("cuda", 0)
+    L, P, Hkv, T, D = 32, 1024, 8, 16, 128
+    chunk = 2 * Hkv * T * D * 2
+    nbytes = L * P * chunk
+    src = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev).normal_()
+    dst = torch.empty_like(src)
+    hb = dkv.dkv_host_alloc_mapped(nbytes // 2, torch.bfloat16)
+    hb.tensor.copy_(src.cpu())
+    res = {}
+    for name, s_ptr in (("hbm_to_hbm", src), ("host_to_hbm", hb.dev_ptr)):
+        for _ in range(args.warmup):
+            dkv.dkv_permute_layout(s_ptr, dst, 0, L, P, chunk)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps = args.steps if name == "hbm_to_hbm" else max(1, args.steps // 10)
+        a.record()
+        for _ in range(steps):
+            dkv.dkv_permute_layout(s_ptr, dst, 0, L, P, chunk)
+        b.record()
+        b.synchronize()
+        ms = a.elapsed_time(b) / steps
+        res[name] = {"ms": ms, "gbs_read": nbytes / (ms * 1e-3) / 1e9}
+    # bit-exact check of the last host -> HBM conversion on sampled chunks
+    v = dst.view(P, L, chunk // 2)
+    s2 = src.view(L, P, chunk // 2)
+    for (l, pp) in ((0, 0), (31, 1023), (7, 512), (20, 3)):
+        assert torch.equal(v[pp, l], s2[l, pp])
+    hb.close()
+    peak, kind = load_peaks()
+    h2d = measure_h2d_peak(dev)
+    hh = res["hbm_to_hbm"]
+    line = {"metric": "block-layout conversion GB/s (layer-first -> page-first, 2 GiB tier)",
+            "value": hh["gbs_read"], "unit": "GB/s (bytes read)", "higher_is_better": True, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "impl": "dkv", "data": "synthetic",
+            "config": {"workload": "layout: L=32, P=1024, Hkv=8, T=16, D=128, bf16 (2 GiB)"},
+            "variants": res,
+            "roofline": {"bound": "hbm", "achieved": 2 * hh["gbs_read"], "peak": peak, "unit": "GB/s",
+                         "frac": 2 * hh["gbs_read"] / peak, "peak_source": kind,
+                         "note": "achieved counts read + write bytes, like the copy peak"},
+            "host_link": {"h2d_peak_gbs": h2d, "host_to_hbm_gbs": res["host_to_hbm"]["gbs_read"],
+                          "frac": res["host_to_hbm"]["gbs_read"] / h2d}}
+    print(json.dumps(line), flush=True)
+
+
+def run_staged_compare(args, cfg, wl, dev):
+    """Conventional offload on the same workload: swap every host-tier block of the step
+    into an HBM staging area (per-block cudaMemcpyAsync, or the GPU copy kernel), then
+    attend over HBM only. Returns per-step times (ms)."""
+    import kv_cache_offload_b200 as dkv
+    lay = wl.lay
+    nh, ns = lay.hbm_blocks, lay.host_blocks
+    tier_elems = cfg.layers * 2 * cfg.Hkv * cfg.T * cfg.D
+    hbm = torch.empty(((nh + ns) * tier_elems,), dtype=torch.bfloat16, device=dev)
+    hbm[: nh * tier_elems].copy_(wl.hbm)
+    pool = dkv.dkv_pool_create(cfg.layers, cfg.Hkv, cfg.D, nh + ns, ns, hbm_base=hbm)
+    out = {}
+    try:
+        dkv.host_tier_tensor(pool).copy_(dkv.host_tier_tensor(wl.pool))
+        table = lay.block_table.clone()
+        table[lay.tier_map == 1] += nh
+        table[lay.block_table < 0] = -1
+        table = table.to(dev)
+        tmap = torch.zeros_like(wl.tmap)
+        src_h = torch.arange(ns, dtype=torch.int32)
+        dst_h = torch.arange(nh, nh + ns, dtype=torch.int32)
+        perm = torch.randperm(ns, generator=torch.Generator().manual_seed(0))
+        ids = {"dma": (src_h[perm].contiguous(), dst_h[perm].contiguous()),
+               "kernel": (src_h.to(dev), dst_h.to(dev))}
+        steps = max(2, min(args.steps, 10))
+        for name, method in (("dma", dkv.DKV_COPY_DMA), ("kernel", dkv.DKV_COPY_KERNEL)):
+            s_ids, d_ids = ids[name]
+
+            def step():
+                dkv.dkv_copy_blocks(pool, 1, 0, s_ids, d_ids, method)
+                dkv.dkv_decode_step(pool, 0, wl.x, wl.W, table, wl.lens, tmap, cfg.Hq, cfg.theta, wl.out, wl.ws)
+
+            step()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(steps):
+                step()
+            b.record()
+            b.synchronize()
+            out["staged_" + name + "_ms"] = a.elapsed_time(b) / steps
+        assert dkv.dkv_check(pool) == dkv.DKV_OK
+        out["staging_hbm_bytes"] = ns * tier_elems * 2
+        out["note"] = ("dma: one cudaMemcpyAsync per block in table order (random physical ids); "
+                       "kernel: one GPU copy kernel; both then attend over HBM only")
+    finally:
+        dkv.dkv_pool_destroy(pool)
+    return out
+
+
 def main():
     args = parse()
+    if args.config == "layout":
+        return run_layout(args)
     if args.config == "gemm":
         rank = int(os.environ.get("RANK", "0"))
         if rank == 0:
@@ -498,15 +618,12 @@ def main():
     e2e_ms = a.elapsed_time(b)
 
     # ---- max over ranks
-    vals = torch.tensor([t_ms, e2e_ms] + stage_ms, dtype=torch.float64, device=dev)
-    if dist:
-        tdist.all_reduce(vals, op=tdist.ReduceOp.MAX)
-    t_ms, e2e_ms = float(vals[0]), float(vals[1])
-    stage_ms = [float(v) for v in vals[2:]]
+    vals = reduce_max_over_ranks([t_ms, e2e_ms] + stage_ms, dist, dev)
+    t_ms, e2e_ms = vals[0], vals[1]
+    stage_ms = vals[2:]
     ms = t_ms / args.steps
-    tokens = cfg.B * world
-    value = tokens / (ms * 1e-3)
-    e2e_val = tokens / (e2e_ms / args.steps * 1e-3)
+    value = replica_throughput(cfg.B, world, ms)
+    e2e_val = replica_throughput(cfg.B, world, e2e_ms / args.steps)
 
     peak, peak_kind = load_peaks()
     attn_ms = stage_ms[1]
@@ -531,17 +648,25 @@ def main():
                    "l2": "inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)},
         "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
         "stage_ms": {"project": stage_ms[0], "attend_and_combine": stage_ms[1]},
-        "roofline": {"bound": "hbm" if not wl.kv_host_bytes else "host_link", "kernel": "attn_splitk_kernel",
-                     "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "peak_source": peak_kind,
-                     "traffic": profiled_traffic(cfg.name),
-                     "algorithmic_bytes_per_launch": wl.kv_bytes},
+        "roofline": ({"bound": "hbm", "kernel": "attn_splitk_kernel",
+                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                      "peak_source": peak_kind,
+                      "traffic": profiled_traffic(cfg.name),
+                      "algorithmic_bytes_per_launch": wl.kv_bytes}
+                     if not wl.kv_host_bytes else
+                     {"bound": "host_link", "kernel": "attn_splitk_kernel",
+                      "achieved": host_info["achieved_gbs"], "peak": host_info["h2d_peak_gbs"], "unit": "GB/s",
+                      "frac": host_info["frac"], "peak_source": "measured cudaMemcpy H2D (pinned, 1 GiB) in this run",
+                      "traffic": None, "algorithmic_bytes_per_launch": wl.kv_host_bytes}),
         "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * args.steps,
         "clocks": clk,
     }
     if host_info:
         line["host_link"] = host_info
+        if args.compare_staged:
+            line["staged_swap_baseline"] = run_staged_compare(args, cfg, wl, dev)
+            line["staged_swap_baseline"]["zero_copy_ms"] = ms
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, 0, args.cpu_seconds)
     if rank == 0:

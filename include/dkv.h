@@ -121,6 +121,23 @@ int dkv_append_kv(dkv_pool* pool, int layer, const uint16_t* k, const uint16_t* 
                   int n_tokens, const int32_t* block_table, int max_blocks,
                   const int32_t* seq_lens, const uint8_t* tier_map, void* stream);
 
+/*
+ * Copy whole blocks between tiers (swap-in / swap-out, "KV Offload" wiki page, sections
+ * Swap-out / Swap-in): for i < n, block src_ids[i] of tier src_tier -> block dst_ids[i] of
+ * tier dst_tier, every layer, K and V, every kv head (bit-exact). Methods:
+ *   DKV_COPY_DMA     one cudaMemcpyAsync per block and layer (runs of consecutive ids on
+ *                    both sides are merged): the copy engine, as conventional offload does;
+ *                    src_ids / dst_ids are HOST arrays.
+ *   DKV_COPY_KERNEL  one kernel whose threads move 16-byte pieces (GPU-assisted I/O,
+ *                    Strata, "「KV Cache 内存层级」系列总纲" §2.4); src_ids / dst_ids are
+ *                    DEVICE arrays; bad ids are skipped and flagged (dkv_check).
+ * The two tiers may be the same (a move within a tier); ranges must not overlap.
+ */
+#define DKV_COPY_DMA    0
+#define DKV_COPY_KERNEL 1
+int dkv_copy_blocks(dkv_pool* pool, int src_tier, int dst_tier, const int32_t* src_ids,
+                    const int32_t* dst_ids, int n, int method, void* stream);
+
 /* Bytes of caller-provided workspace dkv_decode_step needs for this shape. */
 size_t dkv_decode_workspace_bytes(const dkv_pool* pool, int B, int max_blocks,
                                   int num_q_heads, int hidden);

@@ -30,6 +30,8 @@ DKV_TIER_HOST = 1
 DKV_LAYOUT_LAYER_FIRST = 0
 DKV_LAYOUT_PAGE_FIRST = 1
 DKV_HOST_WRITE_COMBINED = 1
+DKV_COPY_DMA = 0
+DKV_COPY_KERNEL = 1
 DKV_GEMM_CPU_AWARE = 0
 DKV_GEMM_NAIVE_ZERO_COPY = 1
 DKV_GEMM_STAGED_SWAP = 2
@@ -79,6 +81,7 @@ _SIGS = {
     "dkv_permute_layout": (_I, [_P, _P, _I, _I, _I64, _I64, _P]),
     "dkv_convert_layout": (_I, [_P, _I, _P, _SZ, _P]),
     "dkv_check": (_I, [_P, _P]),
+    "dkv_copy_blocks": (_I, [_P, _I, _I, _P, _P, _I, _I, _P]),
     "dkv_gemm_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "dkv_host_alloc_mapped": (_I, [_SZ, _I, ctypes.POINTER(_P), ctypes.POINTER(_P)]),
     "dkv_host_free": (_I, [_P]),
@@ -343,6 +346,19 @@ def dkv_gemm(variant: int, A: torch.Tensor, Bt, C: torch.Tensor, workspace: torc
     N = N or C.shape[1]
     _chk(lib().dkv_gemm(variant, _ptr(A), _ptr(Bt), _ptr(C), M, N, K, _ptr(workspace),
                         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def dkv_copy_blocks(pool: int, src_tier: int, dst_tier: int, src_ids: torch.Tensor,
+                    dst_ids: torch.Tensor, method: int = DKV_COPY_KERNEL, stream=None):
+    """Copy blocks between tiers; ids are int32 CPU tensors for DKV_COPY_DMA, CUDA tensors
+    for DKV_COPY_KERNEL."""
+    cuda = method == DKV_COPY_KERNEL
+    _need(src_ids, torch.int32, "src_ids", cuda=cuda)
+    _need(dst_ids, torch.int32, "dst_ids", cuda=cuda)
+    if src_ids.is_cuda != cuda or dst_ids.is_cuda != cuda:
+        raise ValueError("ids must be %s tensors for this method" % ("CUDA" if cuda else "CPU"))
+    _chk(lib().dkv_copy_blocks(pool, src_tier, dst_tier, _ptr(src_ids), _ptr(dst_ids),
+                               src_ids.numel(), method, _stream(stream)))
 
 
 def dkv_check(pool: int, stream=None) -> int:

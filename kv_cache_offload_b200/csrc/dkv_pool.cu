@@ -91,6 +91,42 @@ __global__ void __launch_bounds__(256) permute_chunks_kernel(const uint4* __rest
   }
 }
 
+// Block copy between tiers: item = (block i, layer l, 16-byte piece c); each thread moves
+// four pieces per round so several loads are in flight when the source is host memory.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(PoolView pool, int src_tier, int dst_tier,
+                                                          const int32_t* __restrict__ src_ids,
+                                                          const int32_t* __restrict__ dst_ids, int n) {
+  const int64_t pieces = (int64_t)2 * pool.Hkv * pool.T * pool.D / 8;  // 16-byte pieces per (block, layer)
+  const int64_t per_block = pieces * pool.L;
+  const int64_t total = per_block * n;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; base < total; base += 4 * stride) {
+    uint4 v[4];
+    uint4* dst[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      dst[u] = nullptr;
+      const int64_t it = base + u * stride;
+      if (it >= total) continue;
+      const int i = (int)(it / per_block);
+      const int64_t r = it % per_block;
+      const int l = (int)(r / pieces);
+      const int64_t c = r % pieces;
+      const int64_t s = src_ids[i], d = dst_ids[i];
+      if (s < 0 || s >= tier_blocks(pool, src_tier) || d < 0 || d >= tier_blocks(pool, dst_tier)) {
+        if (c == 0 && l == 0) flag_error(pool.status, kErrBadBlock);
+        continue;
+      }
+      const uint4* src = reinterpret_cast<const uint4*>(tier_base(pool, src_tier) + chunk_offset(pool, src_tier, l, s, 0, 0)) + c;
+      dst[u] = reinterpret_cast<uint4*>(tier_base(pool, dst_tier) + chunk_offset(pool, dst_tier, l, d, 0, 0)) + c;
+      v[u] = __ldcs(src);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (dst[u]) __stcs(dst[u], v[u]);
+  }
+}
+
 }  // namespace dkv
 
 using namespace dkv;
@@ -280,6 +316,45 @@ int dkv_convert_layout(dkv_pool* p, int tier, void* dst, size_t dst_bytes, void*
   const int64_t chunk = (int64_t)2 * p->cfg.num_kv_heads * p->cfg.block_tokens * p->cfg.head_dim * 2;
   const int64_t blocks = tier == DKV_TIER_HBM ? p->cfg.hbm_blocks : p->cfg.host_blocks;
   return dkv_permute_layout(src, dst, p->cfg.layout, p->cfg.num_layers, blocks, chunk, stream);
+}
+
+int dkv_copy_blocks(dkv_pool* p, int src_tier, int dst_tier, const int32_t* src_ids, const int32_t* dst_ids, int n,
+                    int method, void* stream) {
+  if (!p || (n > 0 && (!src_ids || !dst_ids)) || n < 0 || (src_tier != 0 && src_tier != 1) ||
+      (dst_tier != 0 && dst_tier != 1) || (method != DKV_COPY_DMA && method != DKV_COPY_KERNEL))
+    return set_error(DKV_ERR_ARG, "dkv_copy_blocks: bad argument");
+  if (n == 0) return DKV_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  const PoolView v = p->view();
+  const size_t chunk = (size_t)2 * v.Hkv * v.T * v.D * 2;  // one block of one layer, bytes
+  if (method == DKV_COPY_KERNEL) {
+    const int64_t items = (int64_t)n * v.L * (chunk / 16);
+    int64_t grid = (items + 255) / 256;
+    const int64_t cap = (int64_t)p->num_sms * 8;
+    if (grid > cap) grid = cap;
+    copy_blocks_kernel<<<(unsigned)grid, 256, 0, st>>>(v, src_tier, dst_tier, src_ids, dst_ids, n);
+    return cuda_check(cudaGetLastError(), "dkv_copy_blocks kernel");
+  }
+  for (int i = 0; i < n;) {
+    const int64_t s0 = src_ids[i], d0 = dst_ids[i];
+    if (s0 < 0 || s0 >= tier_blocks(v, src_tier) || d0 < 0 || d0 >= tier_blocks(v, dst_tier))
+      return set_error(DKV_ERR_BAD_TABLE, "dkv_copy_blocks: block id out of range at %d", i);
+    int run = 1;  // merge consecutive ids when a block's layers are contiguous (page-first or L == 1)
+    if (v.layout == DKV_LAYOUT_PAGE_FIRST || v.L == 1)
+      while (i + run < n && src_ids[i + run] == s0 + run && dst_ids[i + run] == d0 + run &&
+             s0 + run < tier_blocks(v, src_tier) && d0 + run < tier_blocks(v, dst_tier))
+        ++run;
+    for (int l = 0; l < v.L; ++l) {
+      const size_t bytes = chunk * ((v.layout == DKV_LAYOUT_PAGE_FIRST) ? (size_t)v.L * run : run);
+      const uint16_t* src = tier_base(v, src_tier) + chunk_offset(v, src_tier, l, s0, 0, 0);
+      uint16_t* dst = tier_base(v, dst_tier) + chunk_offset(v, dst_tier, l, d0, 0, 0);
+      int rc = cuda_check(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, st), "dkv_copy_blocks: copy");
+      if (rc) return rc;
+      if (v.layout == DKV_LAYOUT_PAGE_FIRST) break;  // all layers in one copy
+    }
+    i += run;
+  }
+  return DKV_OK;
 }
 
 int dkv_host_alloc_mapped(size_t bytes, int host_flags, void** host_ptr, void** dev_ptr) {
