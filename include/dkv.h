@@ -80,8 +80,9 @@ typedef struct dkv_pool_config {
 typedef struct dkv_tuning {
   int32_t attn_splits;   /* split-K factor of the attention grid (per sequence, kv head) */
   int32_t proj_splits;   /* cluster size of the projection (its reduction split), <= 16 */
-  int32_t attn_variant;  /* attention kernel shape for G = 4: 0 default, 1 deeper ring,
-                            2 two warps per block, 3 both */
+  int32_t attn_variant;  /* attention kernel shape for G = 4: 0 automatic (= 1: q in
+                            registers, 8-stage ring, 3 CTAs/SM), 2 12-stage ring,
+                            3 two warps per block, 5 q in shared memory; (4 is invalid) */
   int32_t attn_lsu_hbm;  /* 1: load HBM-tier blocks with 16-byte cp.async, not bulk copies */
   int32_t reserved[4];
 } dkv_tuning;

@@ -49,7 +49,10 @@ struct AttnCfg {
   static constexpr int SMEM = OFF_BARS + 2 * NST * 8;
   static constexpr int MERGE_BYTES = NCW * HPW * D * 4 + NCW * HPW * 8;
   static_assert(MERGE_BYTES <= NST * STAGE_BYTES, "merge area must fit in the stage ring");
-  static_assert(NST >= kSlots, "ring must hold one block per consumer slot");
+  // Block i uses stage i % NST and consumer slot i % kSlots. Stage loads complete out of
+  // order, and a parity wait is only sound if the stage's barrier is at most one phase
+  // behind the waiter; that holds when every stage belongs to a single slot.
+  static_assert(NST % kSlots == 0, "each stage must belong to exactly one consumer slot");
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -107,10 +110,12 @@ __device__ __forceinline__ void rs_level(float* v, bool up, int mask) {
   }
 }
 
-template <int D, int HPW, int WPB, int NST, int MINB>
+// QS: keep q in shared memory instead of registers (fewer registers, more CTAs per SM).
+template <int D, int HPW, int WPB, int NST, int MINB, bool QS>
 __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
     attn_splitk_kernel(const AttnParams p) {
   using C = AttnCfg<D, HPW, WPB, NST>;
+  constexpr int OFF_Q = (C::SMEM + 15) / 16 * 16;  // q area (QS only): [G][QCH][2][8][4] fp32
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* stages = reinterpret_cast<uint16_t*>(smem);
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
@@ -150,6 +155,7 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
     // broadcast by shuffle, so no dependent global load sits on the per-block path.
     const int64_t rowbase = (int64_t)b * p.max_blocks;
     int pf_tier = 0, pf_phys = 0;
+    int issued = 0;
     for (int i = 0; i < n_local; ++i) {
       if ((i & 31) == 0) {
         const int j = j0 + i + lane;
@@ -178,6 +184,7 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
       if (!valid) {
         mbar_arrive(&full[st]);
         if (lane == 0) mbar_arrive(&full[st]);
+        issued = i + 1;
         continue;
       }
       const uint16_t* kp = tier_base(pool, tier) + chunk_offset(pool, tier, p.layer, phys, 0, g);
@@ -203,8 +210,14 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
         cp_async_arrive_noinc(&full[st]);
         if (lane == 0) mbar_arrive(&full[st]);
       }
+      issued = i + 1;
     }
     cp_async_wait_all();
+    // Never leave with a bulk copy still writing this CTA's shared memory: the last NST
+    // issued loads are the only ones that can be in flight; their stage barrier is at the
+    // load's phase or past it, so the parity wait is exact (bounded, 100 ms).
+    for (int j = issued > NST ? issued - NST : 0; j < issued; ++j)
+      mbar_wait_bounded(&full[j % NST], (j / NST) & 1, pool.status, 100000000ull);
     return;  // consumers below sync only among themselves (named barrier 1)
   }
 
@@ -213,20 +226,32 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
   const int tg = lane >> 3, dg = lane & 7;
   const int hbase = g * C::G + hq * HPW;  // first global q head of this warp
 
-  // q of this lane's key dims, as (even, odd) dim pairs for the packed fp32x2 FMA
-  float2 q2[HPW][C::QCH][4];
-#pragma unroll
-  for (int h = 0; h < HPW; ++h)
-#pragma unroll
-    for (int hh = 0; hh < C::QCH; ++hh) {
-      const float4* src = reinterpret_cast<const float4*>(
-          p.qs + ((int64_t)b * p.Hq + hbase + h) * D + (dg + 8 * hh) * 8);
-      const float4 a = src[0], c = src[1];
-      q2[h][hh][0] = make_float2(a.x, a.y);
-      q2[h][hh][1] = make_float2(a.z, a.w);
-      q2[h][hh][2] = make_float2(c.x, c.y);
-      q2[h][hh][3] = make_float2(c.z, c.w);
+  // q of this lane's key dims, as (even, odd) dim pairs for the packed fp32x2 FMA: in
+  // registers, or (QS) in shared memory laid out [head][hh][half][dg][4] so that the eight
+  // dg lanes read 128 contiguous bytes.
+  float2 q2[QS ? 1 : HPW][QS ? 1 : C::QCH][4];
+  float* qsm = reinterpret_cast<float*>(smem + OFF_Q);
+  if constexpr (QS) {
+    for (int e = threadIdx.x; e < C::G * D; e += C::NCW * 32) {
+      const int h = e / D, d = e % D, c = d / 8, w = d % 8;
+      qsm[(((h * C::QCH + c / 8) * 2 + w / 4) * 8 + c % 8) * 4 + w % 4] =
+          p.qs[((int64_t)b * p.Hq + g * C::G + h) * D + d];
     }
+    named_bar_sync(1, C::NCW * 32);
+  } else {
+#pragma unroll
+    for (int h = 0; h < HPW; ++h)
+#pragma unroll
+      for (int hh = 0; hh < C::QCH; ++hh) {
+        const float4* src = reinterpret_cast<const float4*>(
+            p.qs + ((int64_t)b * p.Hq + hbase + h) * D + (dg + 8 * hh) * 8);
+        const float4 a = src[0], c = src[1];
+        q2[h][hh][0] = make_float2(a.x, a.y);
+        q2[h][hh][1] = make_float2(a.z, a.w);
+        q2[h][hh][2] = make_float2(c.x, c.y);
+        q2[h][hh][3] = make_float2(c.z, c.w);
+      }
+  }
 
   constexpr int NP = C::DPL / 2;  // value-dim pairs per lane
   float2 acc2[HPW][NP];
@@ -253,24 +278,55 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
       float2 v2[C::NV];
 #pragma unroll
       for (int x = 0; x < C::NV; ++x) v2[x] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int i4 = 0; i4 < 4; ++i4) {
-        const int t = tg + 4 * i4;
+      if constexpr (QS) {
 #pragma unroll
         for (int hh = 0; hh < C::QCH; ++hh) {
-          const uint4 w = *reinterpret_cast<const uint4*>(Ks + t * D + (dg + 8 * hh) * 8);
-          const float2 k0 = make_float2(bf16lo(w.x), bf16hi(w.x));
-          const float2 k1 = make_float2(bf16lo(w.y), bf16hi(w.y));
-          const float2 k2 = make_float2(bf16lo(w.z), bf16hi(w.z));
-          const float2 k3 = make_float2(bf16lo(w.w), bf16hi(w.w));
+          float2 kk[4][4];
+#pragma unroll
+          for (int i4 = 0; i4 < 4; ++i4) {
+            const uint4 w = *reinterpret_cast<const uint4*>(Ks + (tg + 4 * i4) * D + (dg + 8 * hh) * 8);
+            kk[i4][0] = make_float2(bf16lo(w.x), bf16hi(w.x));
+            kk[i4][1] = make_float2(bf16lo(w.y), bf16hi(w.y));
+            kk[i4][2] = make_float2(bf16lo(w.z), bf16hi(w.z));
+            kk[i4][3] = make_float2(bf16lo(w.w), bf16hi(w.w));
+          }
 #pragma unroll
           for (int h = 0; h < HPW; ++h) {
-            float2 a = v2[h * 4 + i4];
-            a = __ffma2_rn(q2[h][hh][0], k0, a);
-            a = __ffma2_rn(q2[h][hh][1], k1, a);
-            a = __ffma2_rn(q2[h][hh][2], k2, a);
-            a = __ffma2_rn(q2[h][hh][3], k3, a);
-            v2[h * 4 + i4] = a;
+            const float4* qp = reinterpret_cast<const float4*>(qsm) + (((hq * HPW + h) * C::QCH + hh) * 2) * 8 + dg;
+            const float4 qa = qp[0], qb = qp[8];
+            const float2 q0 = make_float2(qa.x, qa.y), q1 = make_float2(qa.z, qa.w);
+            const float2 q2b = make_float2(qb.x, qb.y), q3 = make_float2(qb.z, qb.w);
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) {
+              float2 a = v2[h * 4 + i4];
+              a = __ffma2_rn(q0, kk[i4][0], a);
+              a = __ffma2_rn(q1, kk[i4][1], a);
+              a = __ffma2_rn(q2b, kk[i4][2], a);
+              a = __ffma2_rn(q3, kk[i4][3], a);
+              v2[h * 4 + i4] = a;
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          const int t = tg + 4 * i4;
+#pragma unroll
+          for (int hh = 0; hh < C::QCH; ++hh) {
+            const uint4 w = *reinterpret_cast<const uint4*>(Ks + t * D + (dg + 8 * hh) * 8);
+            const float2 k0 = make_float2(bf16lo(w.x), bf16hi(w.x));
+            const float2 k1 = make_float2(bf16lo(w.y), bf16hi(w.y));
+            const float2 k2 = make_float2(bf16lo(w.z), bf16hi(w.z));
+            const float2 k3 = make_float2(bf16lo(w.w), bf16hi(w.w));
+#pragma unroll
+            for (int h = 0; h < HPW; ++h) {
+              float2 a = v2[h * 4 + i4];
+              a = __ffma2_rn(q2[h][hh][0], k0, a);
+              a = __ffma2_rn(q2[h][hh][1], k1, a);
+              a = __ffma2_rn(q2[h][hh][2], k2, a);
+              a = __ffma2_rn(q2[h][hh][3], k3, a);
+              v2[h * 4 + i4] = a;
+            }
           }
         }
       }
@@ -451,23 +507,27 @@ __global__ void __launch_bounds__(D) combine_kernel(int Hq, int Hkv, int S,
 
 // ---------------------------------------------------------------------- launchers
 
-template <int D, int HPW, int WPB, int NST, int MINB>
+template <int D, int HPW, int WPB, int NST, int MINB, bool QS = false>
 static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
   using C = AttnCfg<D, HPW, WPB, NST>;
-  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB>;
+  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB, QS>;
+  constexpr int smem = QS ? (C::SMEM + 15) / 16 * 16 + C::G * D * 4 : C::SMEM;
   static bool attr_done = false;  // per instantiation
   if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_check(e, "attention: set smem attribute");
     attr_done = true;
   }
   dim3 grid(p.S, Hkv, B);
-  fn<<<grid, C::THREADS, C::SMEM, st>>>(p);
+  fn<<<grid, C::THREADS, smem, st>>>(p);
   return cuda_check(cudaGetLastError(), "attention launch");
 }
 
-// Kernel shape per (D, G) and variant: 0 = default; 1 = 12-stage ring; 2 = two warps per
-// block with G/2 heads each (G = 4); 3 = both.
+// Kernel shape per (D, G) and variant (G = 4 only; other G have one shape):
+//   0 automatic = 1: q in registers, 8-stage ring, three CTAs per SM
+//   2: 12-stage ring, two CTAs per SM        3: two warps per block (G/2 heads each)
+//   5: q in shared memory, 8-stage ring, three CTAs per SM
+// (Rings must be a multiple of the four consumer slots; see AttnCfg.)
 template <int D>
 static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant, cudaStream_t st) {
   switch (G) {
@@ -475,14 +535,20 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
     case 2: return launch_attn_t<D, 2, 1, 8, 3>(p, B, Hkv, st);
     case 4:
       switch (variant) {
-        case 1: return launch_attn_t<D, 4, 1, 12, 2>(p, B, Hkv, st);
-        case 2: return launch_attn_t<D, 2, 2, 8, 2>(p, B, Hkv, st);
-        case 3: return launch_attn_t<D, 2, 2, 12, 2>(p, B, Hkv, st);
+        case 1: return launch_attn_t<D, 4, 1, 8, 3>(p, B, Hkv, st);
+        case 2: return launch_attn_t<D, 4, 1, 12, 2>(p, B, Hkv, st);
+        case 3: return launch_attn_t<D, 2, 2, 8, 2>(p, B, Hkv, st);
+        case 5: return launch_attn_t<D, 4, 1, 8, 3, true>(p, B, Hkv, st);
         default: return launch_attn_t<D, 4, 1, 8, 3>(p, B, Hkv, st);
       }
     case 8: return launch_attn_t<D, 4, 2, 8, 1>(p, B, Hkv, st);
   }
   return set_error(DKV_ERR_UNSUPPORTED, "attention: unsupported G=%d", G);
+}
+
+int attention_ctas_per_sm(int G, int variant) {
+  (void)G;
+  return variant == 2 || variant == 3 ? 2 : 3;
 }
 
 int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, int variant, cudaStream_t st) {

@@ -67,6 +67,7 @@ struct AttnParams {
 };
 
 int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, int variant, cudaStream_t st);
+int attention_ctas_per_sm(int G, int variant);
 int launch_combine(int B, int Hq, int Hkv, int D, int S, const float2* ml, const float* acc,
                    const float* qs, const float* knew, const float* vnew, uint16_t* out, cudaStream_t st);
 

@@ -200,3 +200,27 @@ def test_staged_calls_match_fused_step():
         assert torch.equal(staged, fused)
     finally:
         ctx.close()
+
+
+@pytest.mark.parametrize("variant", [1, 2, 3, 5])  # 0 (automatic) is 1
+@pytest.mark.parametrize("splits", [1, 0])  # one split: long CTAs that wrap the stage ring
+@pytest.mark.parametrize("D", [64, 128])
+def test_attention_kernel_variants(variant, splits, D):
+    cfg = WL.small_config(B=3, Hq=8, Hkv=2, D=D, H=256, ctx_range=(300, 700), host_prob=0.5)
+    inp = WL.make_decode_inputs(cfg, seed=11)
+    ctx = TL.make_pool(inp)
+    try:
+        base = TL.run_step(ctx, layer=1)
+        dkv.dkv_pool_set_tuning(ctx.pool, attn_splits=splits, attn_variant=variant,
+                                attn_lsu_hbm=variant % 2)
+        x, W = inp.x.cuda(), inp.W.cuda()
+        out = torch.empty_like(base)
+        nws = dkv.dkv_decode_workspace_bytes(ctx.pool, cfg.B, ctx.table.shape[1], cfg.Hq, cfg.H)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        dkv.dkv_decode_step(ctx.pool, 1, x, W, ctx.table, ctx.seq_lens, ctx.tier_map, cfg.Hq, cfg.theta, out, ws)
+        assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
+        TL.assert_out_close(out, TL.oracle_step(inp, layer=1)["out"], "variant %d" % variant)
+        # same splits, same reduction order per (slot, head): the variants agree closely
+        assert (out.float() - base.float()).abs().max().item() <= 2 ** -6
+    finally:
+        ctx.close()
