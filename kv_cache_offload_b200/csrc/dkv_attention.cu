@@ -154,6 +154,13 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
     // Table entries are fetched 32 blocks at a time (lane l holds block base + l) and
     // broadcast by shuffle, so no dependent global load sits on the per-block path.
     const int64_t rowbase = (int64_t)b * p.max_blocks;
+    // chunk address of (phys, K) = kbase[tier] + phys * pstride; the V chunk is kvoff further
+    // (both layouts are linear in the physical id)
+    const int64_t TD = (int64_t)kT * D;
+    const int64_t pstride = (pool.layout == DKV_LAYOUT_LAYER_FIRST ? 2LL : 2LL * pool.L) * pool.Hkv * TD;
+    const int64_t kvoff = (int64_t)pool.Hkv * TD;
+    const uint16_t* kbase0 = pool.tier[0] + chunk_offset(pool, 0, p.layer, 0, 0, g);
+    const uint16_t* kbase1 = pool.tier[1] + chunk_offset(pool, 1, p.layer, 0, 0, g);
     int pf_tier = 0, pf_phys = 0;
     int issued = 0;
     for (int i = 0; i < n_local; ++i) {
@@ -187,8 +194,8 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
         issued = i + 1;
         continue;
       }
-      const uint16_t* kp = tier_base(pool, tier) + chunk_offset(pool, tier, p.layer, phys, 0, g);
-      const uint16_t* vp = tier_base(pool, tier) + chunk_offset(pool, tier, p.layer, phys, 1, g);
+      const uint16_t* kp = (tier ? kbase1 : kbase0) + phys * pstride;
+      const uint16_t* vp = kp + kvoff;
       if (tier == DKV_TIER_HBM && !p.lsu_hbm) {
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
@@ -378,34 +385,39 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
         for (int e = 0; e < NP; ++e) acc2[h][e] = __fmul2_rn(acc2[h][e], a2);
       }
       const int d0 = lane * C::DPL;
-#pragma unroll
-      for (int t = 0; t < kT; ++t) {
-        if (t < ntok) {
-          float2 vf[NP];
-          if constexpr (NP == 2) {
-            const uint2 w = *reinterpret_cast<const uint2*>(Vs + t * D + d0);
-            vf[0] = make_float2(bf16lo(w.x), bf16hi(w.x));
-            vf[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
-          } else {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(Vs + t * D + d0);
-            vf[0] = make_float2(bf16lo(w), bf16hi(w));
-          }
-          float2 pp[HPW];
-          if constexpr (HPW >= 2) {
-#pragma unroll
-            for (int h2 = 0; h2 < HPW; h2 += 2) {
-              const float4 q4 = *reinterpret_cast<const float4*>(pb + t * HPW + h2);
-              pp[h2] = make_float2(q4.x, q4.y);
-              pp[h2 + 1] = make_float2(q4.z, q4.w);
-            }
-          } else {
-            pp[0] = pb[t];
-          }
-#pragma unroll
-          for (int h = 0; h < HPW; ++h)
-#pragma unroll
-            for (int e = 0; e < NP; ++e) acc2[h][e] = __ffma2_rn(pp[h], vf[e], acc2[h][e]);
+      auto pv_token = [&](int t) {
+        float2 vf[NP];
+        if constexpr (NP == 2) {
+          const uint2 w = *reinterpret_cast<const uint2*>(Vs + t * D + d0);
+          vf[0] = make_float2(bf16lo(w.x), bf16hi(w.x));
+          vf[1] = make_float2(bf16lo(w.y), bf16hi(w.y));
+        } else {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(Vs + t * D + d0);
+          vf[0] = make_float2(bf16lo(w), bf16hi(w));
         }
+        float2 pp[HPW];
+        if constexpr (HPW >= 2) {
+#pragma unroll
+          for (int h2 = 0; h2 < HPW; h2 += 2) {
+            const float4 q4 = *reinterpret_cast<const float4*>(pb + t * HPW + h2);
+            pp[h2] = make_float2(q4.x, q4.y);
+            pp[h2 + 1] = make_float2(q4.z, q4.w);
+          }
+        } else {
+          pp[0] = pb[t];
+        }
+#pragma unroll
+        for (int h = 0; h < HPW; ++h)
+#pragma unroll
+          for (int e = 0; e < NP; ++e) acc2[h][e] = __ffma2_rn(pp[h], vf[e], acc2[h][e]);
+      };
+      if (ntok == kT) {  // full block: no per-token tests
+#pragma unroll
+        for (int t = 0; t < kT; ++t) pv_token(t);
+      } else {
+#pragma unroll
+        for (int t = 0; t < kT; ++t)
+          if (t < ntok) pv_token(t);
       }
     }
     __syncwarp();
