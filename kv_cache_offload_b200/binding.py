@@ -14,7 +14,8 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdkv.so")
-HEADER = os.path.join(os.path.dirname(_HERE), "include", "dkv.h")
+INCLUDE = os.path.join(os.path.dirname(_HERE), "include")
+HEADER = os.path.join(INCLUDE, "dkv.h")
 
 DKV_OK = 0
 DKV_ERR_ARG = -1
@@ -36,6 +37,8 @@ DKV_GEMM_CPU_AWARE = 0
 DKV_GEMM_NAIVE_ZERO_COPY = 1
 DKV_GEMM_STAGED_SWAP = 2
 DKV_GEMM_DEVICE = 3
+DKV_PLAN_MAPPED = 0
+DKV_PLAN_HOST = 1
 
 
 class DkvError(RuntimeError):
@@ -57,6 +60,20 @@ class dkv_tuning(ctypes.Structure):
                 ("attn_variant", ctypes.c_int32), ("attn_lsu_hbm", ctypes.c_int32),
                 ("reserved", ctypes.c_int32 * 4)]
 
+
+class dkv_bm_config(ctypes.Structure):
+    _fields_ = [("max_rows", ctypes.c_int32), ("max_blocks", ctypes.c_int32),
+                ("block_tokens", ctypes.c_int32), ("plan_memory", ctypes.c_int32),
+                ("hbm_ids", ctypes.c_int64), ("host_ids", ctypes.c_int64),
+                ("hbm_budget", ctypes.c_int64)]
+
+
+class dkv_layer_io(ctypes.Structure):
+    _fields_ = [("layer", ctypes.c_int32), ("reserved", ctypes.c_int32), ("x", ctypes.c_void_p),
+                ("Wqkv", ctypes.c_void_p), ("out", ctypes.c_void_p)]
+
+
+PLAN_HEADER_BYTES = 32
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -86,6 +103,21 @@ _SIGS = {
     "dkv_host_alloc_mapped": (_I, [_SZ, _I, ctypes.POINTER(_P), ctypes.POINTER(_P)]),
     "dkv_host_free": (_I, [_P]),
     "dkv_gemm": (_I, [_I, _P, _P, _P, _I, _I, _I, _P, _SZ, _P]),
+    "dkv_plan_bytes": (_SZ, [_I, _I]),
+    "dkv_bm_create": (_I, [ctypes.POINTER(dkv_bm_config), ctypes.POINTER(_P)]),
+    "dkv_bm_destroy": (_I, [_P]),
+    "dkv_bm_add": (_I, [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]),
+    "dkv_bm_remove": (_I, [_P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]),
+    "dkv_bm_step": (_I, [_P]),
+    "dkv_bm_rows": (_I, [_P]),
+    "dkv_bm_window": (_I64, [_P]),
+    "dkv_bm_plan": (_I, [_P, _I, ctypes.POINTER(_P), ctypes.POINTER(_P)]),
+    "dkv_bm_tables": (_I, [_P, _P, _P, _P]),
+    "dkv_apply_plan": (_I, [_P, _P, _P, _P, _P, _I, _I, _P]),
+    "dkv_decode_graph_create": (_I, [_P, _P, _I, ctypes.POINTER(dkv_layer_io), _I, _P, _P, _P, _I, _I,
+                                     _I, _I, _F, _P, _SZ, ctypes.POINTER(_P)]),
+    "dkv_graph_launch": (_I, [_P, _P]),
+    "dkv_graph_destroy": (_I, [_P]),
     "dkv_last_error": (ctypes.c_char_p, []),
     "dkv_version": (ctypes.c_char_p, []),
 }
@@ -108,11 +140,15 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-def header_symbols(path: str = HEADER):
-    """Names of the functions include/dkv.h declares."""
-    txt = open(path).read()
-    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    return sorted(set(re.findall(r"\b(dkv_[a-z_0-9]+)\s*\(", txt)))
+def header_symbols(path: Optional[str] = None):
+    """Names of the functions the headers under include/ declare (or one header's)."""
+    import glob
+    paths = [path] if path else sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
+    names = set()
+    for p in paths:
+        txt = re.sub(r"/\*.*?\*/", "", open(p).read(), flags=re.S)
+        names |= set(re.findall(r"\b(dkv_[a-z_0-9]+)\s*\(", txt))
+    return sorted(names)
 
 
 def dkv_last_error() -> str:
@@ -364,3 +400,164 @@ def dkv_copy_blocks(pool: int, src_tier: int, dst_tier: int, src_ids: torch.Tens
 def dkv_check(pool: int, stream=None) -> int:
     """Synchronise and return the pool's status code (DKV_OK or a DKV_ERR_*)."""
     return lib().dkv_check(pool, _stream(stream))
+
+
+# ------------------------------------------------------------ placement and graphs
+
+
+def dkv_plan_bytes(max_rows: int, max_blocks: int) -> int:
+    return lib().dkv_plan_bytes(max_rows, max_blocks)
+
+
+def dkv_bm_create(max_rows: int, max_blocks: int, hbm_ids: int, host_ids: int, hbm_budget: int,
+                  block_tokens: int = 16, plan_memory: int = DKV_PLAN_MAPPED) -> int:
+    cfg = dkv_bm_config(max_rows, max_blocks, block_tokens, plan_memory, hbm_ids, host_ids, hbm_budget)
+    out = _P()
+    _chk(lib().dkv_bm_create(ctypes.byref(cfg), ctypes.byref(out)))
+    return out.value
+
+
+def dkv_bm_destroy(bm: int):
+    _chk(lib().dkv_bm_destroy(bm))
+
+
+def dkv_bm_add(bm: int, seq_len: int) -> int:
+    row = ctypes.c_int32()
+    _chk(lib().dkv_bm_add(bm, seq_len, ctypes.byref(row)))
+    return row.value
+
+
+def dkv_bm_remove(bm: int, row: int) -> int:
+    moved = ctypes.c_int32()
+    _chk(lib().dkv_bm_remove(bm, row, ctypes.byref(moved)))
+    return moved.value
+
+
+def dkv_bm_step(bm: int):
+    _chk(lib().dkv_bm_step(bm))
+
+
+def dkv_bm_rows(bm: int) -> int:
+    r = lib().dkv_bm_rows(bm)
+    if r < 0:
+        raise DkvError(r, dkv_last_error())
+    return r
+
+
+def dkv_bm_window(bm: int) -> int:
+    return lib().dkv_bm_window(bm)
+
+
+def dkv_bm_plan(bm: int, slot: int = -1):
+    """(slot, host address, device alias or None) of a plan buffer."""
+    h, d = _P(), _P()
+    r = lib().dkv_bm_plan(bm, slot, ctypes.byref(h), ctypes.byref(d))
+    if r < 0:
+        raise DkvError(r, dkv_last_error())
+    return r, h.value, d.value
+
+
+def dkv_bm_tables(bm: int, max_rows: int, max_blocks: int):
+    """Host snapshot (block_table int32, tier_map uint8, seq_lens int32) as numpy arrays."""
+    import numpy as np
+    bt = np.empty((max_rows, max_blocks), np.int32)
+    tm = np.empty((max_rows, max_blocks), np.uint8)
+    sl = np.empty((max_rows,), np.int32)
+    _chk(lib().dkv_bm_tables(bm, bt.ctypes.data, tm.ctypes.data, sl.ctypes.data))
+    return bt, tm, sl
+
+
+def read_plan(host_addr: int):
+    """Decode a plan buffer at a host address into {"moves", "entries", "seq_lens"} lists
+    (tuples of ints), for inspection and tests."""
+    import numpy as np
+    hdr = np.ctypeslib.as_array((ctypes.c_int32 * 8).from_address(host_addr))
+    n_moves, n_entries, n_rows, _, move_cap, entry_cap, _, _ = [int(v) for v in hdr]
+    base = host_addr + PLAN_HEADER_BYTES
+    mv = np.ctypeslib.as_array((ctypes.c_int32 * (4 * max(n_moves, 1))).from_address(base))
+    en = np.ctypeslib.as_array((ctypes.c_int32 * (4 * max(n_entries, 1))).from_address(base + 16 * move_cap))
+    sl = np.ctypeslib.as_array((ctypes.c_int32 * max(n_rows, 1)).from_address(base + 16 * (move_cap + entry_cap)))
+    return {"moves": [tuple(int(v) for v in mv[4 * i:4 * i + 4]) for i in range(n_moves)],
+            "entries": [tuple(int(v) for v in en[4 * i:4 * i + 4]) for i in range(n_entries)],
+            "seq_lens": [int(v) for v in sl[:n_rows]]}
+
+
+class BlockManager:
+    """The library's block manager (dkv_bm_*): recency-window placement over the two tiers.
+    Each operation writes a plan; `plan()` gives its device alias for dkv_apply_plan or a
+    decode graph."""
+
+    def __init__(self, max_rows: int, max_blocks: int, hbm_ids: int, host_ids: int, hbm_budget: int,
+                 block_tokens: int = 16, plan_memory: int = DKV_PLAN_MAPPED):
+        self.max_rows, self.max_blocks = max_rows, max_blocks
+        self.handle = dkv_bm_create(max_rows, max_blocks, hbm_ids, host_ids, hbm_budget, block_tokens,
+                                    plan_memory)
+
+    def add(self, seq_len: int) -> int:
+        return dkv_bm_add(self.handle, seq_len)
+
+    def remove(self, row: int) -> int:
+        return dkv_bm_remove(self.handle, row)
+
+    def step(self):
+        dkv_bm_step(self.handle)
+
+    @property
+    def rows(self) -> int:
+        return dkv_bm_rows(self.handle)
+
+    @property
+    def window(self) -> int:
+        return dkv_bm_window(self.handle)
+
+    def plan(self, slot: int = -1):
+        return dkv_bm_plan(self.handle, slot)
+
+    def last_plan(self):
+        return read_plan(self.plan()[1])
+
+    def tables(self):
+        return dkv_bm_tables(self.handle, self.max_rows, self.max_blocks)
+
+    def close(self):
+        if self.handle:
+            dkv_bm_destroy(self.handle)
+            self.handle = 0
+
+
+def dkv_apply_plan(pool: int, plan_dev: int, block_table: torch.Tensor, tier_map: torch.Tensor,
+                   seq_lens: torch.Tensor, stream=None):
+    _need(block_table, torch.int32, "block_table"); _need(tier_map, torch.uint8, "tier_map")
+    _need(seq_lens, torch.int32, "seq_lens")
+    R, MB = block_table.shape
+    _chk(lib().dkv_apply_plan(pool, plan_dev, _ptr(block_table), _ptr(tier_map), _ptr(seq_lens), R, MB,
+                              _stream(stream)))
+
+
+def dkv_decode_graph_create(pool: int, plan_dev: Optional[int], layers, block_table: torch.Tensor,
+                            seq_lens: torch.Tensor, tier_map: torch.Tensor, B: int, hidden: int,
+                            num_q_heads: int, rope_theta: float, workspace: torch.Tensor) -> int:
+    """layers: sequence of (layer, x, Wqkv, out) with x [B, hidden], out [B, Hq*D] (bf16).
+    block_table / tier_map are the full [max_rows, max_blocks] device tables; the step
+    decodes rows 0..B-1."""
+    _need(block_table, torch.int32, "block_table"); _need(tier_map, torch.uint8, "tier_map")
+    _need(seq_lens, torch.int32, "seq_lens")
+    arr = (dkv_layer_io * len(layers))()
+    for i, (layer, x, W, out) in enumerate(layers):
+        _need(x, torch.bfloat16, "x"); _need(W, torch.bfloat16, "Wqkv"); _need(out, torch.bfloat16, "out")
+        arr[i] = dkv_layer_io(layer, 0, _ptr(x), _ptr(W), _ptr(out))
+    R, MB = block_table.shape
+    g = _P()
+    _chk(lib().dkv_decode_graph_create(pool, plan_dev, R, arr, len(layers), _ptr(block_table), _ptr(seq_lens),
+                                       _ptr(tier_map), B, MB, hidden, num_q_heads, float(rope_theta),
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                       ctypes.byref(g)))
+    return g.value
+
+
+def dkv_graph_launch(graph: int, stream=None):
+    _chk(lib().dkv_graph_launch(graph, _stream(stream)))
+
+
+def dkv_graph_destroy(graph: int):
+    _chk(lib().dkv_graph_destroy(graph))

@@ -1,6 +1,6 @@
 """Build libdkv.so in-tree for sm_100a with nvcc (no JIT cache, no torch extension).
 
-Each csrc/*.cu is compiled to an object under <repo>/_build/ in parallel, then linked into
+Each csrc/*.cu and csrc/*.cpp (host-only C++) is compiled to an object under <repo>/_build/ in parallel, then linked into
 kv_cache_offload_b200/libdkv.so. Rebuilds only when a source or header is newer than the
 library.
 """
@@ -32,7 +32,7 @@ def _nvcc() -> str:
 
 
 def _sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def _deps():

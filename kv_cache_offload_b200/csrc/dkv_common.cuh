@@ -16,6 +16,7 @@ enum : int {
   kErrBadBlock = 2,
   kErrCtxTooLong = 4,
   kErrTimeout = 8,
+  kErrBadPlan = 16,
 };
 
 // What a kernel needs to address the pool.

@@ -395,9 +395,10 @@ int dkv_check(dkv_pool* p, void* stream) {
   cudaMemset(p->d_status, 0, sizeof(int));
   if (word & kErrTimeout)
     return set_error(DKV_ERR_TIMEOUT, "device wait timed out (status 0x%x)", word);
-  return set_error(DKV_ERR_BAD_TABLE, "device rejected table entries (status 0x%x:%s%s%s)", word,
+  return set_error(DKV_ERR_BAD_TABLE, "device rejected table entries (status 0x%x:%s%s%s%s)", word,
                    (word & kErrBadTier) ? " bad-tier" : "", (word & kErrBadBlock) ? " bad-block-id" : "",
-                   (word & kErrCtxTooLong) ? " context-exceeds-table" : "");
+                   (word & kErrCtxTooLong) ? " context-exceeds-table" : "",
+                   (word & kErrBadPlan) ? " plan-header-mismatch" : "");
 }
 
 }  // extern "C"

@@ -44,3 +44,10 @@ def test_error_paths_without_device():
 def test_struct_layout_matches_header():
     assert ctypes.sizeof(dkv.binding.dkv_pool_config) == 48
     assert ctypes.sizeof(dkv.binding.dkv_tuning) == 32
+
+
+def test_placement_structs_match_header():
+    assert ctypes.sizeof(dkv.binding.dkv_bm_config) == 40
+    assert ctypes.sizeof(dkv.binding.dkv_layer_io) == 32
+    assert dkv.dkv_plan_bytes(3, 5) == 32 + 15 * 32 + 3 * 4
+    assert dkv.dkv_plan_bytes(0, 5) == 0
