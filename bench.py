@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="dkv", choices=["dkv", "reference"])
-    ap.add_argument("--config", default="8b_hbm", choices=sorted(WL.CONFIGS) + ["gemm", "layout"])
+    ap.add_argument("--config", default="8b_hbm", choices=sorted(WL.CONFIGS) + ["gemm", "layout", "adaptive"])
     ap.add_argument("--compare-staged", action="store_true",
                     help="host-tier configs: also time swap-in (DMA and copy kernel) + HBM attention")
     ap.add_argument("--attn-splits", type=int, default=0)
@@ -507,10 +507,168 @@ def run_staged_compare(args, cfg, wl, dev):
     return out
 
 
+class AdaptiveModel:
+    """L layers of the 8B-shaped decode step over one pool, with the library's block manager
+    placing each sequence's blocks (newest budget/B in HBM, the rest in the host tier) and
+    one CUDA graph per plan buffer replaying plan application + every layer's step."""
+
+    def __init__(self, dkv, dev, L, B, ctx, budget, headroom_tokens, seed=0):
+        self.dkv, self.L, self.B, self.ctx = dkv, L, B, ctx
+        H, Hq, Hkv, D, T = 4096, 32, 8, 128, 16
+        self.H, self.Hq, self.Hkv, self.D, self.T, self.theta = H, Hq, Hkv, D, T, 5e5
+        self.max_blocks = (ctx + headroom_tokens) // T + 1
+        self.budget = budget
+        hbm_ids = budget + B + 1
+        host_ids = max(B * (ctx // T + 1) - budget, 0) + B * (headroom_tokens // T + 2)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(seed)
+        blk = L * 2 * Hkv * T * D
+        self.hbm = gpu_randn_bf16((hbm_ids * blk,), gen)
+        self.pool = dkv.dkv_pool_create(L, Hkv, D, hbm_ids, host_ids, hbm_base=self.hbm)
+        # host tier: random HBM blocks copied over the link by the library's copy kernel
+        dst = torch.arange(host_ids, dtype=torch.int32, device=dev)
+        dkv.dkv_copy_blocks(self.pool, 0, 1, (dst % hbm_ids).to(torch.int32).contiguous(), dst,
+                            dkv.DKV_COPY_KERNEL)
+        self.W = [gpu_randn_bf16(((Hq + 2 * Hkv) * D, H), gen, std=1.0 / math.sqrt(H)) for _ in range(L)]
+        self.x = [gpu_randn_bf16((B, H), gen) for _ in range(L)]
+        self.out = [torch.empty((B, Hq * D), dtype=torch.bfloat16, device=dev) for _ in range(L)]
+        self.bt = torch.zeros((B, self.max_blocks), dtype=torch.int32, device=dev)
+        self.tm = torch.zeros((B, self.max_blocks), dtype=torch.uint8, device=dev)
+        self.sl = torch.zeros((B,), dtype=torch.int32, device=dev)
+        self.bm = dkv.BlockManager(B, self.max_blocks, hbm_ids, host_ids, budget)
+        for _ in range(B):
+            self.bm.add(ctx)
+            dkv.dkv_apply_plan(self.pool, self.bm.plan()[2], self.bt, self.tm, self.sl)
+        torch.cuda.current_stream().synchronize()
+        self.check_tables()
+        nws = dkv.dkv_decode_workspace_bytes(self.pool, B, self.max_blocks, Hq, H)
+        self.ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+        layers = [(l, self.x[l], self.W[l], self.out[l]) for l in range(L)]
+        self.graphs = [dkv.dkv_decode_graph_create(self.pool, self.bm.plan(s)[2], layers, self.bt, self.sl,
+                                                   self.tm, B, H, Hq, self.theta, self.ws) for s in (0, 1)]
+        self.layers = layers
+        if dkv.dkv_check(self.pool) != dkv.DKV_OK:  # synchronises: no plan buffer is still being read
+            raise RuntimeError("adaptive setup: " + dkv.dkv_last_error())
+
+    def check_tables(self):
+        """The device tables must equal the manager's snapshot on every cached block."""
+        bt, tm, sl = self.bm.tables()
+        dbt, dtm, dsl = self.bt.cpu().numpy(), self.tm.cpu().numpy(), self.sl.cpu().numpy()
+        for b in range(self.B):
+            nb = int(sl[b]) // self.T + 1
+            if int(dsl[b]) != int(sl[b]) or (dbt[b, :nb] != bt[b, :nb]).any() or (dtm[b, :nb] != tm[b, :nb]).any():
+                raise RuntimeError("device tables differ from the block manager's (row %d)" % b)
+
+    def bytes_per_step(self):
+        """Algorithmic bytes of one L-layer step at the current placement: cached KV by tier
+        (K and V of every cached token, every kv head, every layer) and W of every layer."""
+        bt, tm, sl = self.bm.tables()
+        per_tok = 2 * self.Hkv * self.D * 2 * self.L
+        hbm = host = 0
+        for b in range(self.B):
+            c = int(sl[b])
+            for j in range((c + self.T - 1) // self.T):
+                n = min(self.T, c - j * self.T)
+                if tm[b, j]:
+                    host += n * per_tok
+                else:
+                    hbm += n * per_tok
+        return hbm, host, self.L * (self.Hq + 2 * self.Hkv) * self.D * self.H * 2
+
+    def run(self, steps, warmup, graph=True):
+        """Time `steps` serving steps (host: count the last tokens, write a plan; device:
+        apply it and decode every layer) after `warmup`; returns ms per step (CUDA events)."""
+        dkv = self.dkv
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for i in range(warmup + steps):
+            if i == warmup:
+                a.record()
+            self.bm.step()  # waits until the device released the plan buffer it rewrites
+            slot, _, plan_dev = self.bm.plan()
+            if graph:
+                dkv.dkv_graph_launch(self.graphs[slot])
+            else:
+                dkv.dkv_apply_plan(self.pool, plan_dev, self.bt, self.tm, self.sl)
+                for (l, x, W, out) in self.layers:
+                    dkv.dkv_decode_step(self.pool, l, x, W, self.bt, self.sl, self.tm, self.Hq, self.theta, out,
+                                        self.ws)
+        b.record()
+        b.synchronize()
+        rc = dkv.dkv_check(self.pool)
+        if rc != dkv.DKV_OK:
+            raise RuntimeError("adaptive run: " + dkv.dkv_last_error())
+        self.check_tables()
+        return a.elapsed_time(b) / steps
+
+    def close(self):
+        for g in self.graphs:
+            self.dkv.dkv_graph_destroy(g)
+        self.bm.close()
+        self.dkv.dkv_pool_destroy(self.pool)
+
+
+def run_adaptive(args):
+    """Adaptive placement (hot blocks in HBM, cold blocks read in place from the host tier)
+    over a 4-layer slice of the 8B-shaped model, B=16 x 32768 cached tokens (8 GiB of KV),
+    across HBM budgets; and CUDA-graph replay vs eager launches of a 32-layer step."""
+    import kv_cache_offload_b200 as dkv
+    from kv_cache_offload_b200.build import build
+    build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, kind = load_peaks()
+    h2d = measure_h2d_peak(dev)
+    L, B, ctx = 4, 16, 32768
+    total = B * (ctx // 16 + 1)
+    steps = max(2, min(args.steps, 6))
+    warm = max(3, min(args.warmup, 3))
+    sweep = []
+    for frac in (1.0, 0.5, 0.25, 1.0 / 16, 0.0):
+        budget = int(round(frac * total))
+        m = AdaptiveModel(dkv, dev, L, B, ctx, budget, headroom_tokens=16 * 4)
+        try:
+            ms = m.run(steps, warm, graph=True)
+            ms_eager = m.run(steps, 1, graph=False)
+            hbm_b, host_b, w_b = m.bytes_per_step()
+            t_roof = max((hbm_b + w_b) / (peak * 1e9), host_b / (h2d * 1e9)) * 1e3
+            sweep.append({"hbm_frac": frac, "budget_blocks": budget, "window_blocks": m.bm.window,
+                          "ms_per_step": ms, "tokens_per_s": B / (ms * 1e-3), "eager_ms_per_step": ms_eager,
+                          "kv_hbm_bytes": hbm_b, "kv_host_bytes": host_b, "w_bytes": w_b,
+                          "hbm_tier_bytes": m.hbm.numel() * 2, "t_roof_ms": t_roof, "frac_of_roofline": t_roof / ms})
+        finally:
+            m.close()
+        torch.cuda.empty_cache()
+    # launch overhead: a full-depth (32-layer) step on short contexts, all in HBM
+    Lg, ctxg = 32, 2048
+    m = AdaptiveModel(dkv, dev, Lg, B, ctxg, B * ((ctxg + 16 * 8) // 16 + 1), headroom_tokens=16 * 8)
+    try:
+        ms_g = m.run(50, warm, graph=True)
+        ms_e = m.run(50, warm, graph=False)
+        hbm_b, host_b, w_b = m.bytes_per_step()
+        graph = {"layers": Lg, "batch": B, "cached_tokens": ctxg, "graph_ms_per_step": ms_g,
+                 "eager_ms_per_step": ms_e, "speedup": ms_e / ms_g,
+                 "t_roof_ms": (hbm_b + w_b) / (peak * 1e9) * 1e3,
+                 "frac_of_roofline_graph": (hbm_b + w_b) / (peak * 1e9) * 1e3 / ms_g}
+    finally:
+        m.close()
+    best = sweep[0]
+    line = {"metric": "adaptive placement: 4-layer decode step tokens/s vs HBM budget", "value": best["tokens_per_s"],
+            "unit": "tokens/s", "higher_is_better": True, "n_gpus": 1, "steps": steps, "warmup": warm,
+            "impl": "dkv", "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "8B-shaped layers x4, B=16, 32768 cached tokens each, 16-token blocks; "
+                                   "recency-window placement at HBM budget fractions 1, 1/2, 1/4, 1/16, 0; "
+                                   "each step = host plan + one graph replay (plan apply + 4 layers)"},
+            "h2d_peak_gbs": h2d, "hbm_peak_gbs": peak, "peak_source": kind,
+            "sweep": sweep, "graph_vs_eager": graph}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.config == "layout":
         return run_layout(args)
+    if args.config == "adaptive":
+        return run_adaptive(args)
     if args.config == "gemm":
         rank = int(os.environ.get("RANK", "0"))
         if rank == 0:

@@ -56,7 +56,8 @@ typedef struct dkv_plan_header {
   int32_t move_cap;
   int32_t entry_cap;
   int32_t max_rows;
-  int32_t reserved;
+  int32_t applied;     /* 0 while the plan is pending; dkv_apply_plan sets it to 1 once the
+                          device has finished reading the buffer */
 } dkv_plan_header;
 
 typedef struct dkv_plan_move { int32_t src_tier, src_id, dst_tier, dst_id; } dkv_plan_move;
@@ -77,14 +78,20 @@ typedef struct dkv_bm_config {
   int64_t host_ids;      /* host-tier physical ids the manager may use: 0..host_ids-1 */
   int64_t hbm_budget;    /* blocks kept in HBM at rest, 0 <= budget; when budget > 0,
                             hbm_ids >= budget + 1 (one id of headroom for a step) */
+  int32_t wait_ms;       /* longest wait for a plan buffer to be released (0 = 10000) */
+  int32_t reserved;      /* 0 */
 } dkv_bm_config;
 
 typedef struct dkv_bm dkv_bm;  /* opaque block manager (host-side state, plan buffers) */
 
 /*
  * Create a block manager with no sequences. It holds two plan buffers: operation k writes
- * buffer k mod 2, so a caller may prepare the next plan while the device applies the last
- * one, but must not start operation k+2 before the device finished reading plan k.
+ * buffer k mod 2, so the host prepares plan k+1 while the device applies plan k. Every
+ * plan must be applied, in order, from the buffer's device alias (dkv_apply_plan or a
+ * decode graph holding it). Under DKV_PLAN_MAPPED an operation first waits until the
+ * device has released the buffer it is about to rewrite (the header's `applied` word,
+ * set by the apply kernel); after wait_ms it fails with DKV_ERR_TIMEOUT and changes
+ * nothing. Under DKV_PLAN_HOST there is no wait: the caller moves plans itself.
  * Errors: DKV_ERR_ARG (bad config), DKV_ERR_OOM (plan buffers), DKV_ERR_CUDA.
  */
 int dkv_bm_create(const dkv_bm_config* cfg, dkv_bm** out);
@@ -92,8 +99,9 @@ int dkv_bm_destroy(dkv_bm* bm);
 
 /*
  * Placement operations (see the policy above). Each writes a plan into the next plan
- * buffer. On error (DKV_ERR_ARG, or DKV_ERR_CAPACITY when a tier has too few free ids
- * or the table too few rows or columns) the manager and the plan buffers are unchanged.
+ * buffer. On error (DKV_ERR_ARG; DKV_ERR_CAPACITY when a tier has too few free ids or
+ * the table too few rows or columns; DKV_ERR_TIMEOUT when the buffer was not released)
+ * the manager and the plan buffers are unchanged.
  *   dkv_bm_add:    *row receives the new sequence's table row (= the old row count).
  *   dkv_bm_remove: *moved_from receives the old row of the sequence now at `row`, or -1
  *                  when `row` was the last row (the caller moves its per-row inputs).
@@ -126,7 +134,10 @@ int dkv_bm_tables(const dkv_bm* bm, int32_t* block_table, uint8_t* tier_map, int
  * device copy), copies the moved blocks between the pool's tiers, and writes the device
  * tables (block_table int32 / tier_map uint8 [max_rows][max_blocks], seq_lens int32
  * [max_rows]). The counts are read on the device, so the launch can sit in a CUDA graph
- * and be replayed with new plans written to the same buffer. A plan whose header does not
+ * and be replayed with new plans written to the same buffer. When the device has finished
+ * reading the plan, the kernel sets the header's `applied` word (the buffer must be
+ * host-visible and writable: a mapped plan buffer's device alias). Launches on one pool
+ * must not overlap (they share a completion counter). A plan whose header does not
  * match max_rows / max_blocks, or whose moves or entries name a bad tier or id, is skipped
  * or partly skipped and flagged in the pool's status word (dkv_check: DKV_ERR_BAD_TABLE).
  */

@@ -65,7 +65,7 @@ class dkv_bm_config(ctypes.Structure):
     _fields_ = [("max_rows", ctypes.c_int32), ("max_blocks", ctypes.c_int32),
                 ("block_tokens", ctypes.c_int32), ("plan_memory", ctypes.c_int32),
                 ("hbm_ids", ctypes.c_int64), ("host_ids", ctypes.c_int64),
-                ("hbm_budget", ctypes.c_int64)]
+                ("hbm_budget", ctypes.c_int64), ("wait_ms", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class dkv_layer_io(ctypes.Structure):
@@ -410,8 +410,8 @@ def dkv_plan_bytes(max_rows: int, max_blocks: int) -> int:
 
 
 def dkv_bm_create(max_rows: int, max_blocks: int, hbm_ids: int, host_ids: int, hbm_budget: int,
-                  block_tokens: int = 16, plan_memory: int = DKV_PLAN_MAPPED) -> int:
-    cfg = dkv_bm_config(max_rows, max_blocks, block_tokens, plan_memory, hbm_ids, host_ids, hbm_budget)
+                  block_tokens: int = 16, plan_memory: int = DKV_PLAN_MAPPED, wait_ms: int = 0) -> int:
+    cfg = dkv_bm_config(max_rows, max_blocks, block_tokens, plan_memory, hbm_ids, host_ids, hbm_budget, wait_ms, 0)
     out = _P()
     _chk(lib().dkv_bm_create(ctypes.byref(cfg), ctypes.byref(out)))
     return out.value
@@ -488,10 +488,10 @@ class BlockManager:
     decode graph."""
 
     def __init__(self, max_rows: int, max_blocks: int, hbm_ids: int, host_ids: int, hbm_budget: int,
-                 block_tokens: int = 16, plan_memory: int = DKV_PLAN_MAPPED):
+                 block_tokens: int = 16, plan_memory: int = DKV_PLAN_MAPPED, wait_ms: int = 0):
         self.max_rows, self.max_blocks = max_rows, max_blocks
         self.handle = dkv_bm_create(max_rows, max_blocks, hbm_ids, host_ids, hbm_budget, block_tokens,
-                                    plan_memory)
+                                    plan_memory, wait_ms)
 
     def add(self, seq_len: int) -> int:
         return dkv_bm_add(self.handle, seq_len)

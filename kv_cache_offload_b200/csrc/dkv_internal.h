@@ -19,7 +19,7 @@ struct dkv_pool {
   uint16_t* host_h;   // host-side address of the host tier
   uint16_t* host_d;   // device alias of the host tier
   size_t host_bytes;
-  int* d_status;
+  int* d_status;      // device scratch: [0] status word, [32] plan-apply CTA counter
   dkv_tuning tuning;
 
   dkv::PoolView view() const {
@@ -39,6 +39,9 @@ struct dkv_pool {
 };
 
 namespace dkv {
+
+constexpr int kPoolScratchInts = 64;
+constexpr int kApplyCounterIdx = 32;
 
 int set_error(int code, const char* fmt, ...);
 int cuda_check(cudaError_t e, const char* what);

@@ -14,9 +14,12 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <functional>
 #include <new>
 #include <queue>
+#include <thread>
 #include <vector>
 
 #include "../../include/dkv_placement.h"
@@ -107,6 +110,23 @@ struct dkv_bm {
     moves.push_back({DKV_TIER_HOST, (int32_t)old, DKV_TIER_HBM, (int32_t)nw});
     touch(r, j);
   }
+  // Wait until the device released the buffer the next plan goes to (mapped plans only).
+  int wait_released() const {
+    if (cfg.plan_memory != DKV_PLAN_MAPPED) return DKV_OK;
+    volatile int32_t* applied = &reinterpret_cast<dkv_plan_header*>(plan_h[next_slot])->applied;
+    if (!*applied) {
+      const int ms = cfg.wait_ms > 0 ? cfg.wait_ms : 10000;
+      const auto t0 = std::chrono::steady_clock::now();
+      while (!*applied) {
+        if (std::chrono::steady_clock::now() - t0 > std::chrono::milliseconds(ms))
+          return set_error(DKV_ERR_TIMEOUT, "dkv_bm: plan buffer %d still holds an unapplied plan after %d ms",
+                           next_slot, ms);
+        std::this_thread::yield();
+      }
+    }
+    std::atomic_thread_fence(std::memory_order_acquire);
+    return DKV_OK;
+  }
   // Write the plan under construction into the next buffer.
   void finish() {
     uint8_t* p = plan_h[next_slot];
@@ -131,7 +151,8 @@ struct dkv_bm {
     h.move_cap = (int32_t)cap;
     h.entry_cap = (int32_t)cap;
     h.max_rows = cfg.max_rows;
-    h.reserved = 0;
+    h.applied = 0;
+    std::atomic_thread_fence(std::memory_order_release);
     *reinterpret_cast<dkv_plan_header*>(p) = h;
     last_slot = next_slot;
     next_slot ^= 1;
@@ -152,7 +173,7 @@ int dkv_bm_create(const dkv_bm_config* c, dkv_bm** out) {
   if (!c || !out) return set_error(DKV_ERR_ARG, "dkv_bm_create: null argument");
   *out = nullptr;
   if (c->max_rows < 1 || c->max_blocks < 1 || c->block_tokens < 1 || c->hbm_ids < 0 || c->host_ids < 0 ||
-      c->hbm_budget < 0 || c->hbm_ids > INT32_MAX || c->host_ids > INT32_MAX ||
+      c->hbm_budget < 0 || c->hbm_ids > INT32_MAX || c->host_ids > INT32_MAX || c->wait_ms < 0 ||
       (c->plan_memory != DKV_PLAN_MAPPED && c->plan_memory != DKV_PLAN_HOST))
     return set_error(DKV_ERR_ARG, "dkv_bm_create: bad configuration");
   if (c->hbm_budget > 0 && c->hbm_ids < c->hbm_budget + 1)
@@ -204,6 +225,7 @@ int dkv_bm_create(const dkv_bm_config* c, dkv_bm** out) {
     h->max_blocks = c->max_blocks;
     h->max_rows = c->max_rows;
     h->move_cap = h->entry_cap = c->max_rows * c->max_blocks;
+    h->applied = 1;  // nothing pending: the first operations need not wait
   }
   *out = bm;
   return DKV_OK;
@@ -235,6 +257,7 @@ int dkv_bm_add(dkv_bm* bm, int32_t seq_len, int32_t* row) {
   if (bm->free_ids[DKV_TIER_HOST].size() < demote + (nb - hot) ||
       bm->free_ids[DKV_TIER_HBM].size() + demote < hot)
     return set_error(DKV_ERR_CAPACITY, "dkv_bm_add: not enough free blocks");
+  if (int rc = bm->wait_released()) return rc;
   bm->begin();
   for (int r = 0; r < bm->n; ++r)
     while (bm->hbm[r] > W) bm->demote_oldest(r);
@@ -256,6 +279,7 @@ int dkv_bm_add(dkv_bm* bm, int32_t seq_len, int32_t* row) {
 
 int dkv_bm_remove(dkv_bm* bm, int32_t row, int32_t* moved_from) {
   if (!bm || row < 0 || row >= bm->n) return set_error(DKV_ERR_ARG, "dkv_bm_remove: bad row");
+  if (int rc = bm->wait_released()) return rc;
   bm->begin();
   const int32_t nb = bm->nb_of(bm->len[row]);
   for (int j = 0; j < nb; ++j) {
@@ -308,6 +332,7 @@ int dkv_bm_step(dkv_bm* bm) {
   }
   if (bm->free_ids[DKV_TIER_HOST].size() < host_need)
     return set_error(DKV_ERR_CAPACITY, "dkv_bm_step: not enough free host blocks");
+  if (int rc = bm->wait_released()) return rc;
   bm->begin();
   for (int r = 0; r < bm->n; ++r) {
     bm->len[r] += 1;

@@ -8,6 +8,8 @@
 // "「KV Cache 内存层级」系列总纲", §2.1 DirectKV and §五, names the dynamic addresses of
 // staged copies as what keeps offload from CUDA-graph replay); the graph below holds the
 // plan's application and every layer's decode step.
+#include <stddef.h>
+
 #include <new>
 
 #include "dkv_internal.h"
@@ -19,24 +21,15 @@ namespace dkv {
 // 16-byte pieces, four loads in flight per thread (the source may be host memory read over
 // the host link). Then every thread takes table entries and cached-token counts.
 // Plan words are read with ld.global.cv: the host rewrites the buffer between launches.
-__global__ void __launch_bounds__(256) apply_plan_kernel(PoolView pool, const uint8_t* __restrict__ plan,
-                                                         int32_t* __restrict__ table,
-                                                         uint8_t* __restrict__ tier_map,
-                                                         int32_t* __restrict__ seq_lens, int max_rows,
-                                                         int max_blocks) {
-  __shared__ int4 s_hdr[2];
-  __shared__ int4 s_move;
-  if (threadIdx.x < 2) s_hdr[threadIdx.x] = __ldcv(reinterpret_cast<const int4*>(plan) + threadIdx.x);
-  __syncthreads();
-  const int n_moves = s_hdr[0].x, n_entries = s_hdr[0].y, n_rows = s_hdr[0].z;
-  const int move_cap = s_hdr[1].x, entry_cap = s_hdr[1].y;
-  const int64_t cap = (int64_t)max_rows * max_blocks;
-  if (s_hdr[0].w != max_blocks || s_hdr[1].z != max_rows || move_cap != cap || entry_cap != cap ||
-      n_moves < 0 || n_moves > move_cap || n_entries < 0 || n_entries > entry_cap || n_rows < 0 ||
-      n_rows > max_rows) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(pool.status, kErrBadPlan);
-    return;
-  }
+// The last CTA to finish (a counter in the pool's device scratch, reset by that CTA) sets
+// the header's `applied` word in the plan buffer, which tells the block manager that the
+// buffer may be rewritten.
+__device__ __forceinline__ void apply_plan_body(const PoolView& pool, const uint8_t* plan, const int4 h0,
+                                                const int4 h1, int4& s_move, int32_t* __restrict__ table,
+                                                uint8_t* __restrict__ tier_map, int32_t* __restrict__ seq_lens,
+                                                int max_rows, int max_blocks) {
+  const int n_moves = h0.x, n_entries = h0.y, n_rows = h0.z;
+  const int move_cap = h1.x, entry_cap = h1.y;
   const int4* moves = reinterpret_cast<const int4*>(plan + sizeof(dkv_plan_header));
   const int4* entries = moves + move_cap;
   const int32_t* lens = reinterpret_cast<const int32_t*>(entries + entry_cap);
@@ -84,11 +77,41 @@ __global__ void __launch_bounds__(256) apply_plan_kernel(PoolView pool, const ui
   for (int64_t i = gt; i < n_rows; i += gs) seq_lens[i] = __ldcv(lens + i);
 }
 
+__global__ void __launch_bounds__(256) apply_plan_kernel(PoolView pool, uint8_t* plan, int32_t* __restrict__ table,
+                                                         uint8_t* __restrict__ tier_map,
+                                                         int32_t* __restrict__ seq_lens, int max_rows,
+                                                         int max_blocks, int* done_ctr) {
+  __shared__ int4 s_hdr[2];
+  __shared__ int4 s_move;
+  if (threadIdx.x < 2) s_hdr[threadIdx.x] = __ldcv(reinterpret_cast<const int4*>(plan) + threadIdx.x);
+  __syncthreads();
+  const int4 h0 = s_hdr[0], h1 = s_hdr[1];
+  const int64_t cap = (int64_t)max_rows * max_blocks;
+  const bool ok = h0.w == max_blocks && h1.z == max_rows && h1.x == cap && h1.y == cap && h0.x >= 0 &&
+                  h0.x <= h1.x && h0.y >= 0 && h0.y <= h1.y && h0.z >= 0 && h0.z <= max_rows;
+  if (ok)
+    apply_plan_body(pool, plan, h0, h1, s_move, table, tier_map, seq_lens, max_rows, max_blocks);
+  else if (blockIdx.x == 0 && threadIdx.x == 0)
+    flag_error(pool.status, kErrBadPlan);
+
+  __syncthreads();  // every read of the plan by this CTA is done
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(done_ctr, 1) == (int)gridDim.x - 1) {
+      *done_ctr = 0;  // the next launch (stream-ordered) starts from zero
+      __threadfence_system();
+      *reinterpret_cast<volatile int32_t*>(plan + offsetof(dkv_plan_header, applied)) = 1;
+      __threadfence_system();
+    }
+  }
+}
+
 static int launch_apply_plan(const dkv_pool* p, const void* plan, int32_t* table, uint8_t* tier_map,
                              int32_t* seq_lens, int max_rows, int max_blocks, cudaStream_t st) {
   // Fixed grid (the plan's size is only known on the device): one CTA per SM.
-  apply_plan_kernel<<<p->num_sms, 256, 0, st>>>(p->view(), static_cast<const uint8_t*>(plan), table, tier_map,
-                                                seq_lens, max_rows, max_blocks);
+  apply_plan_kernel<<<p->num_sms, 256, 0, st>>>(p->view(), static_cast<uint8_t*>(const_cast<void*>(plan)), table,
+                                                tier_map, seq_lens, max_rows, max_blocks,
+                                                p->d_status + kApplyCounterIdx);
   return cuda_check(cudaGetLastError(), "dkv_apply_plan kernel");
 }
 

@@ -210,8 +210,8 @@ int dkv_pool_create(const dkv_pool_config* cfg, dkv_pool** out) {
     p->host_h = static_cast<uint16_t*>(h);
     p->host_d = static_cast<uint16_t*>(d);
   }
-  e = cudaMalloc(&p->d_status, sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, sizeof(int));
+  e = cudaMalloc(&p->d_status, kPoolScratchInts * sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(p->d_status, 0, kPoolScratchInts * sizeof(int));
   if (e != cudaSuccess) {
     if (p->host_h) cudaFreeHost(p->host_h);
     if (p->own_hbm) cudaFree(p->hbm);

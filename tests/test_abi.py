@@ -47,7 +47,7 @@ def test_struct_layout_matches_header():
 
 
 def test_placement_structs_match_header():
-    assert ctypes.sizeof(dkv.binding.dkv_bm_config) == 40
+    assert ctypes.sizeof(dkv.binding.dkv_bm_config) == 48
     assert ctypes.sizeof(dkv.binding.dkv_layer_io) == 32
     assert dkv.dkv_plan_bytes(3, 5) == 32 + 15 * 32 + 3 * 4
     assert dkv.dkv_plan_bytes(0, 5) == 0

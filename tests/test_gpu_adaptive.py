@@ -307,3 +307,32 @@ def test_apply_plan_rejects_bad_plans():
         assert int(lp.bt[0, 0]) == int(before[0][0, 0])
     finally:
         lp.close()
+
+
+def test_manager_waits_for_the_device_to_release_a_plan_buffer():
+    """Operation k rewrites plan buffer k mod 2 only after the device applied plan k-2;
+    otherwise it times out and changes nothing."""
+    lp = Loop(0, 64, 2, max_rows=2, max_blocks=6, budget=2)
+    try:
+        lp.bm.close()
+        lp.bm = dkv.BlockManager(2, 6, lp.hbm_ids, lp.host_ids, 2, wait_ms=200)
+        lp.bm.add(20)                                   # plan 0 -> buffer 0
+        dkv.dkv_apply_plan(lp.pool, lp.bm.plan()[2], lp.bt, lp.tm, lp.sl)
+        lp.bm.step()                                    # plan 1 -> buffer 1, not applied yet
+        lp.bm.step()                                    # plan 2 -> buffer 0 (waits for plan 0: applied)
+        snap = lp.bm.tables()
+        with pytest.raises(dkv.DkvError) as e:
+            lp.bm.step()                                # buffer 1 still holds plan 1
+        assert e.value.code == dkv.DKV_ERR_TIMEOUT
+        for a, b in zip(snap, lp.bm.tables()):
+            assert np.array_equal(a, b)
+        for slot in (1, 0):                             # apply plans 1 and 2, in order
+            dkv.dkv_apply_plan(lp.pool, lp.bm.plan(slot)[2], lp.bt, lp.tm, lp.sl)
+        lp.bm.step()                                    # now proceeds
+        dkv.dkv_apply_plan(lp.pool, lp.bm.plan()[2], lp.bt, lp.tm, lp.sl)
+        assert dkv.dkv_check(lp.pool) == dkv.DKV_OK
+        bt, tm, sl = lp.bm.tables()
+        assert int(lp.sl[0]) == int(sl[0]) == 23
+        assert torch.equal(lp.bt[0, :2].cpu(), torch.from_numpy(bt[0, :2]))
+    finally:
+        lp.close()
