@@ -160,8 +160,8 @@ size_t dkv_decode_workspace_bytes(const dkv_pool* pool, int B, int max_blocks,
  * out: device [B][Hq*D] bf16. workspace: device, >= dkv_decode_workspace_bytes(...),
  * 256-byte aligned; its contents need no initialisation.
  * Supported: 1 <= B <= 32, hidden % 64 == 0, Hq % Hkv == 0 with Hq/Hkv in {1,2,4,8}.
- * Three stream-ordered kernels (projection, attention, combine); no host synchronisation,
- * no allocation, so the call can be captured into a CUDA graph.
+ * Two stream-ordered kernels (projection; attention with the split combine fused); no host
+ * synchronisation, no allocation, so the call can be captured into a CUDA graph.
  */
 int dkv_decode_step(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t* Wqkv,
                     const int32_t* block_table, const int32_t* seq_lens,
