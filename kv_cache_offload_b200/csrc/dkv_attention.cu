@@ -7,22 +7,33 @@
 //  * one CTA per (split s, kv head g, sequence b) walks a contiguous range of logical
 //    blocks; the KV of kv head g is read once for all G = Hq/Hkv query heads;
 //  * one producer warp fills an NST-stage shared-memory ring, one stage per block
-//    (K chunk [T][D] then V chunk [T][D], both contiguous in the pool):
-//      - HBM-tier block: one lane issues two bulk copies (TMA engine) of the chunks;
+//    (K rows [T][D] then V rows [T][D]):
+//      - HBM-tier block: bulk copies (TMA engine) of the chunks, issued by the lanes;
 //      - host-tier block: all 32 lanes issue 16-byte cp.async loads straight from the
 //        mapped pinned host memory (coalesced 512-byte warp requests), no staging buffer;
 //    both complete on the stage's mbarrier, so the consumers see one kind of stage;
-//  * four consumer "slots" (WPB warps each; heads split across the WPB warps) take
-//    blocks round robin, each keeping its own online-softmax state (running max m,
-//    running sum l, accumulator acc) in registers; the slots merge at the end and the CTA
-//    writes one partial state (m, l, acc[D]) per q head to the workspace.
+//  * four consumer "slots" take blocks round robin, each keeping its own online-softmax
+//    state (running max m, running sum l, accumulator) in registers; the slots merge at
+//    the end and the CTA writes one partial state (m, l, acc[D]) per q head to the
+//    workspace; the last split CTA of a (sequence, kv head) merges the splits.
 //
-// Scores are computed in the log2 domain: q arrives pre-scaled by log2(e)/sqrt(D), so
-// p = 2^(s - m). Arithmetic is fp32 on CUDA cores (a decode query is a handful of rows:
-// G flops per byte of KV, HBM-bound, not a tensor-core contraction).
+// Scores are in the log2 domain: q arrives pre-scaled by log2(e)/sqrt(D), so p = 2^(s - m).
+// Two consumer implementations:
+//  * tensor cores (default): per block, S = Q.K^T and O^T += V^T.P^T as m16n8k16 bf16
+//    mma.sync with fp32 accumulation. The G query rows of a kv head are padded to the
+//    16-row tile, and the spare rows carry the bf16 low parts: q = q_hi + q_lo (rows
+//    0..G-1 and 8..8+G-1) and p = p_hi + p_lo (separate columns), so the products keep
+//    about 16 significant bits of the fp32 q and p. A decode step is HBM-bound at G
+//    flops per KV byte; the tensor cores are used because they turn ~800 issued
+//    instructions per block into ~100, which is what kept the CUDA-core version from
+//    the memory roofline. Stages use the TMA 128-byte swizzle, so ldmatrix is conflict-free.
+//  * CUDA cores (variant 1 and the older tunings): packed fp32x2 FMAs.
+#include <cuda_bf16.h>
 #include <math.h>
+#include <string.h>
 
 #include "dkv_internal.h"
+#include "dkv_umma.cuh"
 
 namespace dkv {
 
@@ -110,6 +121,175 @@ __device__ __forceinline__ void rs_level(float* v, bool up, int mask) {
   }
 }
 
+// ------------------------------------------------------------- slot merge + combine
+// The consumer slots have left their state in shared memory: acc [NCW*HPW][D] fp32 at the
+// base, then (m, l) per (warp, head). Merge the kSlots slots per q head, write this
+// split's partial state, and, when the launch fuses the combine, let the last split CTA of
+// (b, g) merge all S partial states in split order with the new token's term.
+template <int D, int HPW, int WPB>
+__device__ __forceinline__ void attn_merge_combine(const AttnParams& p, uint8_t* smem, int b, int g, int s,
+                                                   int warp, int lane) {
+  constexpr int G = HPW * WPB;
+  constexpr int NCW = kSlots * WPB;
+  const PoolView& pool = p.pool;
+  const float* macc = reinterpret_cast<const float*>(smem);
+  const float2* mml = reinterpret_cast<const float2*>(smem + NCW * HPW * D * 4);
+  for (int o = threadIdx.x; o < G * D; o += NCW * 32) {
+    const int hh = o / D, d = o % D;
+    const int wq = hh / HPW, h = hh % HPW;
+    float M = -INFINITY;
+#pragma unroll
+    for (int sl = 0; sl < kSlots; ++sl) M = fmaxf(M, mml[(sl * WPB + wq) * HPW + h].x);
+    float A = 0.f, Ls = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int sl = 0; sl < kSlots; ++sl) {
+        const float2 ml = mml[(sl * WPB + wq) * HPW + h];
+        const float w = fast_exp2(ml.x - M);
+        A = fmaf(macc[((sl * WPB + wq) * HPW + h) * D + d], w, A);
+        Ls = fmaf(ml.y, w, Ls);
+      }
+    }
+    const int64_t base = ((int64_t)b * p.Hq + g * G + hh) * p.S + s;
+    p.part_acc[base * D + d] = A;
+    if (d == 0) p.part_ml[base] = make_float2(M, Ls);
+  }
+
+  // fused combine: the last split CTA of (b, g) to finish merges all S partial states
+  // (in split order, so the result does not depend on which CTA finishes last)
+  if (p.out) {
+    __shared__ int s_last;
+    __shared__ float s_new[8];
+    __threadfence();
+    named_bar_sync(1, NCW * 32);
+    if (threadIdx.x == 0) s_last = atomicAdd(p.cnt + (int64_t)b * pool.Hkv + g, 1) == p.S - 1;
+    named_bar_sync(1, NCW * 32);
+    if (s_last) {
+      __threadfence();
+      const float* kn = p.knew + ((int64_t)b * pool.Hkv + g) * D;
+      for (int hh = warp; hh < G; hh += NCW) {
+        const float sc = new_token_score(p.qs + ((int64_t)b * p.Hq + g * G + hh) * D, kn, D, lane);
+        if (lane == 0) s_new[hh] = sc;
+      }
+      named_bar_sync(1, NCW * 32);
+      for (int o = threadIdx.x; o < G * D; o += NCW * 32) {
+        const int hh = o / D, d = o % D;
+        const int hg = g * G + hh;
+        const float r = combine_value(p.part_ml, p.part_acc, p.S, ((int64_t)b * p.Hq + hg) * p.S, D, d,
+                                      s_new[hh], p.vnew[((int64_t)b * pool.Hkv + g) * D + d]);
+        p.out[((int64_t)b * p.Hq + hg) * D + d] = f32_to_bf16_bits(r);
+      }
+      if (threadIdx.x == 0) p.cnt[(int64_t)b * pool.Hkv + g] = 0;
+    }
+  }
+}
+
+// ------------------------------------------------------------------- producer warp
+// Fills the NST-stage ring for blocks j0..j1-1 of (b, g). A stage holds the K rows then the
+// V rows of one block, in one of two layouts:
+//   packed (SW = false): row r of K at byte r*2D, of V at (T + r)*2D; HBM blocks arrive by
+//     two bulk copies (one per chunk);
+//   swizzled (SW = true): per chunk, D/64 boxes of [T rows][128 bytes] (dims 64h..64h+63),
+//     the 16-byte piece c of row r stored at piece c ^ (r mod 8) (the TMA 128-byte
+//     swizzle; the stage is 1024-byte aligned); HBM blocks arrive by 2*D/64 TMA tensor
+//     copies through `tmap` (the HBM tier as [rows][D]).
+// Host-tier blocks (and HBM blocks when p.lsu_hbm) arrive by 16-byte cp.async from all 32
+// lanes into the same layout. Table entries are fetched 32 blocks at a time (lane l holds
+// block base + l) and broadcast by shuffle, so no dependent global load sits on the
+// per-block path.
+template <int D, int NST, bool SW>
+__device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensorMap* tmap, uint8_t* stages,
+                                             int* flags, uint64_t* full, uint64_t* empty, int b, int g, int ctx,
+                                             int j0, int j1, int lane) {
+  constexpr int DATA_BYTES = 2 * kT * D * 2;
+  constexpr int CHUNK = kT * D * 2;  // bytes of the K (or V) rows of one block
+  const PoolView& pool = p.pool;
+  const int n_local = j1 - j0;
+  const int64_t rowbase = (int64_t)b * p.max_blocks;
+  // chunk address of (phys, K) = kbase[tier] + phys * pstride; the V chunk is kvoff further
+  // (both layouts are linear in the physical id)
+  const int64_t TD = (int64_t)kT * D;
+  const int64_t pstride = (pool.layout == DKV_LAYOUT_LAYER_FIRST ? 2LL : 2LL * pool.L) * pool.Hkv * TD;
+  const int64_t kvoff = (int64_t)pool.Hkv * TD;
+  const uint16_t* kbase0 = pool.tier[0] + chunk_offset(pool, 0, p.layer, 0, 0, g);
+  const uint16_t* kbase1 = pool.tier[1] + chunk_offset(pool, 1, p.layer, 0, 0, g);
+  int pf_tier = 0, pf_phys = 0;
+  int issued = 0;
+  for (int i = 0; i < n_local; ++i) {
+    if ((i & 31) == 0) {
+      const int j = j0 + i + lane;
+      if (j < j1) {
+        pf_tier = p.tier_map[rowbase + j];
+        pf_phys = p.table[rowbase + j];
+      }
+    }
+    const int st = i % NST;
+    const int k = i / NST;
+    if (k > 0 && !mbar_wait_bounded(&empty[st], (k - 1) & 1, pool.status)) break;
+    const int j = j0 + i;
+    const int tier = __shfl_sync(0xffffffffu, pf_tier, i & 31);
+    const int64_t phys = __shfl_sync(0xffffffffu, pf_phys, i & 31);
+    const int ntok = min(kT, ctx - j * kT);
+    bool valid = true;
+    if (tier > 1) {
+      valid = false;
+      if (lane == 0) flag_error(pool.status, kErrBadTier);
+    } else if (phys < 0 || phys >= tier_blocks(pool, tier)) {
+      valid = false;
+      if (lane == 0) flag_error(pool.status, kErrBadBlock);
+    }
+    uint8_t* dst = stages + st * DATA_BYTES;
+    if (lane == 0) flags[st] = valid ? ntok : -1;
+    if (!valid) {
+      mbar_arrive(&full[st]);
+      if (lane == 0) mbar_arrive(&full[st]);
+      issued = i + 1;
+      continue;
+    }
+    const uint16_t* kp = (tier ? kbase1 : kbase0) + phys * pstride;
+    const uint16_t* vp = kp + kvoff;
+    if (tier == DKV_TIER_HBM && !p.lsu_hbm) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[st], DATA_BYTES);
+        mbar_arrive(&full[st]);
+        if constexpr (SW) {
+          const int row = (int)((kp - pool.tier[0]) / D);  // row of the [rows][D] tier view
+#pragma unroll
+          for (int kv = 0; kv < 2; ++kv)
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+              tma_load_2d(dst + kv * CHUNK + h * kT * 128, tmap, 64 * h, row + kv * (int)(kvoff / D), &full[st]);
+        } else {
+          bulk_g2s(dst, kp, CHUNK, &full[st]);
+          bulk_g2s(dst + CHUNK, vp, CHUNK, &full[st]);
+        }
+      } else {
+        mbar_arrive(&full[st]);
+      }
+    } else {
+      constexpr int RP = 2 * D / 16;       // 16-byte pieces per row
+      constexpr int PIECES = 2 * kT * RP;  // per stage
+#pragma unroll
+      for (int c = 0; c < PIECES / 32; ++c) {
+        const int idx = c * 32 + lane;
+        const int kv = idx / (kT * RP), r = (idx / RP) % kT, q = idx % RP;
+        const int off = SW ? kv * CHUNK + (q >> 3) * kT * 128 + r * 128 + (((q & 7) ^ (r & 7)) << 4)
+                           : kv * CHUNK + r * 2 * D + q * 16;
+        cp_async16(dst + off, (kv ? vp : kp) + r * D + q * 8);
+      }
+      cp_async_arrive_noinc(&full[st]);
+      if (lane == 0) mbar_arrive(&full[st]);
+    }
+    issued = i + 1;
+  }
+  cp_async_wait_all();
+  // Never leave with a bulk copy still writing this CTA's shared memory: the last NST
+  // issued loads are the only ones that can be in flight; their stage barrier is at the
+  // load's phase or past it, so the parity wait is exact (bounded, 100 ms).
+  for (int j = issued > NST ? issued - NST : 0; j < issued; ++j)
+    mbar_wait_bounded(&full[j % NST], (j / NST) & 1, pool.status, 100000000ull);
+}
+
 // QS: keep q in shared memory instead of registers (fewer registers, more CTAs per SM).
 template <int D, int HPW, int WPB, int NST, int MINB, bool QS>
 __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
@@ -150,81 +330,7 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
   __syncthreads();
 
   if (warp == C::NCW) {
-    // ------------------------------------------------------------------ producer
-    // Table entries are fetched 32 blocks at a time (lane l holds block base + l) and
-    // broadcast by shuffle, so no dependent global load sits on the per-block path.
-    const int64_t rowbase = (int64_t)b * p.max_blocks;
-    // chunk address of (phys, K) = kbase[tier] + phys * pstride; the V chunk is kvoff further
-    // (both layouts are linear in the physical id)
-    const int64_t TD = (int64_t)kT * D;
-    const int64_t pstride = (pool.layout == DKV_LAYOUT_LAYER_FIRST ? 2LL : 2LL * pool.L) * pool.Hkv * TD;
-    const int64_t kvoff = (int64_t)pool.Hkv * TD;
-    const uint16_t* kbase0 = pool.tier[0] + chunk_offset(pool, 0, p.layer, 0, 0, g);
-    const uint16_t* kbase1 = pool.tier[1] + chunk_offset(pool, 1, p.layer, 0, 0, g);
-    int pf_tier = 0, pf_phys = 0;
-    int issued = 0;
-    for (int i = 0; i < n_local; ++i) {
-      if ((i & 31) == 0) {
-        const int j = j0 + i + lane;
-        if (j < j1) {
-          pf_tier = p.tier_map[rowbase + j];
-          pf_phys = p.table[rowbase + j];
-        }
-      }
-      const int st = i % NST;
-      const int k = i / NST;
-      if (k > 0 && !mbar_wait_bounded(&empty[st], (k - 1) & 1, pool.status)) break;
-      const int j = j0 + i;
-      const int tier = __shfl_sync(0xffffffffu, pf_tier, i & 31);
-      const int64_t phys = __shfl_sync(0xffffffffu, pf_phys, i & 31);
-      const int ntok = min(kT, ctx - j * kT);
-      bool valid = true;
-      if (tier > 1) {
-        valid = false;
-        if (lane == 0) flag_error(pool.status, kErrBadTier);
-      } else if (phys < 0 || phys >= tier_blocks(pool, tier)) {
-        valid = false;
-        if (lane == 0) flag_error(pool.status, kErrBadBlock);
-      }
-      uint16_t* dst = stages + st * C::STAGE_ELEMS;
-      if (lane == 0) flags[st] = valid ? ntok : -1;
-      if (!valid) {
-        mbar_arrive(&full[st]);
-        if (lane == 0) mbar_arrive(&full[st]);
-        issued = i + 1;
-        continue;
-      }
-      const uint16_t* kp = (tier ? kbase1 : kbase0) + phys * pstride;
-      const uint16_t* vp = kp + kvoff;
-      if (tier == DKV_TIER_HBM && !p.lsu_hbm) {
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[st], C::STAGE_BYTES);
-          mbar_arrive(&full[st]);
-          bulk_g2s(dst, kp, C::STAGE_BYTES / 2, &full[st]);
-          bulk_g2s(dst + kT * D, vp, C::STAGE_BYTES / 2, &full[st]);
-        } else {
-          mbar_arrive(&full[st]);
-        }
-      } else {
-        constexpr int PIECES = C::STAGE_BYTES / 16;  // 16-byte pieces per stage
-        constexpr int HALF = PIECES / 2;
-#pragma unroll
-        for (int c = 0; c < PIECES / 32; ++c) {
-          const int idx = c * 32 + lane;
-          const uint16_t* src = idx < HALF ? kp + idx * 8 : vp + (idx - HALF) * 8;
-          cp_async16(dst + idx * 8, src);
-        }
-        cp_async_arrive_noinc(&full[st]);
-        if (lane == 0) mbar_arrive(&full[st]);
-      }
-      issued = i + 1;
-    }
-    cp_async_wait_all();
-    // Never leave with a bulk copy still writing this CTA's shared memory: the last NST
-    // issued loads are the only ones that can be in flight; their stage barrier is at the
-    // load's phase or past it, so the parity wait is exact (bounded, 100 ms).
-    for (int j = issued > NST ? issued - NST : 0; j < issued; ++j)
-      mbar_wait_bounded(&full[j % NST], (j / NST) & 1, pool.status, 100000000ull);
+    attn_produce<D, NST, false>(p, nullptr, smem, flags, full, empty, b, g, ctx, j0, j1, lane);
     return;  // consumers below sync only among themselves (named barrier 1)
   }
 
@@ -442,54 +548,259 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
   if (head_leader) mml[warp * HPW + h_lane] = make_float2(m_run, l_tot);
   named_bar_sync(1, C::NCW * 32);
 
-  for (int o = threadIdx.x; o < C::G * D; o += C::NCW * 32) {
-    const int hh = o / D, d = o % D;
-    const int wq = hh / HPW, h = hh % HPW;
-    float M = -INFINITY;
+  attn_merge_combine<D, HPW, WPB>(p, smem, b, g, s, warp, lane);
+}
+
+// ------------------------------------------------------------ tensor-core consumer
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
+// c (16x8 fp32) += a (16x16 bf16, row) . b (16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// (x, y) -> bf16 pairs hi = rn(x, y) and lo = rn((x, y) - hi); the low half holds x.
+__device__ __forceinline__ void split_bf16x2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x - hf.x, y - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// One consumer warp per slot, all G query heads of kv head g. Fragment layouts are those
+// of mma.m16n8k16 (lane = 4*grp + qd):
+//   S tile (rows = q rows, cols = 8 tokens): A = q rows (hi part of head h in row h, lo part
+//   in row 8 + h), B = K rows via ldmatrix; the lane gets S_hi and S_lo of head grp for
+//   tokens 2qd, 2qd+1 in c0..c3 and adds them in place.
+//   O^T tile (rows = 16 value dims, cols = 8): A = V^T via ldmatrix.trans, B = P^T, whose
+//   fragment is exactly what the lane holds after the softmax (head grp, tokens 2qd, 2qd+1,
+//   2qd+8, 2qd+9). Columns: G = 8 uses two tiles (p_hi, p_lo); G <= 4 puts p_hi of head c
+//   in column c and p_lo in column 4 + c (taken from lane ^ 16).
+template <int D, int G, int NST, int MINB>
+__global__ void __launch_bounds__((kSlots + 1) * 32, MINB)
+    attn_mma_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap) {
+  constexpr int STAGE = 2 * kT * D * 2;  // swizzled K and V rows of one block
+  constexpr int CHUNK = kT * D * 2;
+  constexpr int NCW = kSlots;
+  constexpr int KS = D / 16;
+  constexpr int NTP = G == 8 ? 2 : 1;
+  constexpr int OFF_FLAGS = NST * STAGE;
+  constexpr int OFF_BARS = (OFF_FLAGS + NST * 4 + 7) / 8 * 8;
+  static_assert(NST % kSlots == 0, "each stage must belong to exactly one consumer slot");
+  static_assert(NCW * G * D * 4 + NCW * G * 8 <= NST * STAGE, "merge area must fit in the stage ring");
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  // the 128-byte swizzle is a function of address bits 4..9: stages start 1024-byte aligned
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  int* flags = reinterpret_cast<int*>(smem + OFF_FLAGS);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BARS);
+  uint64_t* empty = full + NST;
+
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const PoolView& pool = p.pool;
+
+  int ctx = p.seq_lens[b];
+  if (ctx < 0 || ctx / kT + 1 > p.max_blocks) {
+    if (threadIdx.x == 0 && s == 0 && g == 0) flag_error(pool.status, kErrCtxTooLong);
+    ctx = ctx < 0 ? 0 : min(ctx, p.max_blocks * kT);
+  }
+  const int nb = (ctx + kT - 1) / kT;
+  const int j0 = (int)((int64_t)nb * s / p.S);
+  const int j1 = (int)((int64_t)nb * (s + 1) / p.S);
+  const int n_local = j1 - j0;
+
+  if (threadIdx.x == 0) {
 #pragma unroll
-    for (int sl = 0; sl < kSlots; ++sl) M = fmaxf(M, mml[(sl * WPB + wq) * HPW + h].x);
-    float A = 0.f, Ls = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int sl = 0; sl < kSlots; ++sl) {
-        const float2 ml = mml[(sl * WPB + wq) * HPW + h];
-        const float w = fast_exp2(ml.x - M);
-        A = fmaf(macc[((sl * WPB + wq) * HPW + h) * D + d], w, A);
-        Ls = fmaf(ml.y, w, Ls);
-      }
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&full[i], 33);  // 32 producer lanes + 1 flag publish
+      mbar_init(&empty[i], 1);  // lane 0 of the consuming warp
     }
-    const int64_t base = ((int64_t)b * p.Hq + g * C::G + hh) * p.S + s;
-    p.part_acc[base * D + d] = A;
-    if (d == 0) p.part_ml[base] = make_float2(M, Ls);
+    mbar_fence_init();
+  }
+  __syncthreads();
+
+  if (warp == NCW) {
+    attn_produce<D, NST, true>(p, &tmap, smem, flags, full, empty, b, g, ctx, j0, j1, lane);
+    return;
   }
 
-  // ---- fused combine: the last split CTA of (b, g) to finish merges all S partial states
-  // (in split order, so the result does not depend on which CTA finishes last)
-  if (p.out) {
-    __shared__ int s_last;
-    __shared__ float s_new[8];
-    __threadfence();
-    named_bar_sync(1, C::NCW * 32);
-    if (threadIdx.x == 0) s_last = atomicAdd(p.cnt + (int64_t)b * pool.Hkv + g, 1) == p.S - 1;
-    named_bar_sync(1, C::NCW * 32);
-    if (s_last) {
-      __threadfence();
-      const float* kn = p.knew + ((int64_t)b * pool.Hkv + g) * D;
-      for (int hh = warp; hh < C::G; hh += C::NCW) {
-        const float sc = new_token_score(p.qs + ((int64_t)b * p.Hq + g * C::G + hh) * D, kn, D, lane);
-        if (lane == 0) s_new[hh] = sc;
-      }
-      named_bar_sync(1, C::NCW * 32);
-      for (int o = threadIdx.x; o < C::G * D; o += C::NCW * 32) {
-        const int hh = o / D, d = o % D;
-        const int hg = g * C::G + hh;
-        const float r = combine_value(p.part_ml, p.part_acc, p.S, ((int64_t)b * p.Hq + hg) * p.S, D, d,
-                                      s_new[hh], p.vnew[((int64_t)b * pool.Hkv + g) * D + d]);
-        p.out[((int64_t)b * p.Hq + hg) * D + d] = f32_to_bf16_bits(r);
-      }
-      if (threadIdx.x == 0) p.cnt[(int64_t)b * pool.Hkv + g] = 0;
+  const int slot = warp;
+  const int grp = lane >> 2, qd = lane & 3;
+  constexpr unsigned FULL = 0xffffffffu;
+
+  // q of head grp as A fragments: rows grp (hi) and grp + 8 (lo), dims 16ks + 2qd + {0,1,8,9}
+  uint32_t qa[KS][4];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) qa[ks][0] = qa[ks][1] = qa[ks][2] = qa[ks][3] = 0u;
+  if (grp < G) {
+    const float* q = p.qs + ((int64_t)b * p.Hq + g * G + grp) * D;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const float2 x0 = *reinterpret_cast<const float2*>(q + 16 * ks + 2 * qd);
+      const float2 x1 = *reinterpret_cast<const float2*>(q + 16 * ks + 2 * qd + 8);
+      split_bf16x2(x0.x, x0.y, qa[ks][0], qa[ks][1]);
+      split_bf16x2(x1.x, x1.y, qa[ks][2], qa[ks][3]);
     }
   }
+
+  float o[KS][NTP][4];
+#pragma unroll
+  for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NTP; ++nt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;  // head grp (rows >= G carry zeros)
+
+  const uint32_t sbase = smem_u32(smem);
+  // ldmatrix row addresses in the swizzled stage (piece c of row r at c ^ (r & 7)):
+  //   K (non-trans): row = token lane&7 (+8 nt), pieces of dims 32*k2 + 8*(lane>>3);
+  //   V (trans):     row = token 8*(lane>>4) + (lane&7), pieces of dims 16*mt + 8*((lane>>3)&1)
+  const int r7 = lane & 7;
+  const uint32_t krow = r7 * 128;
+  const uint32_t kx0 = (((lane >> 3) ^ r7) << 4), kx1 = (((4 + (lane >> 3)) ^ r7) << 4);
+  const uint32_t vrow = CHUNK + (8 * (lane >> 4) + r7) * 128;
+  const int vb = (lane >> 3) & 1;
+  // the heads whose rescale factor applies to this lane's two O^T columns
+  const int hc0 = G == 8 ? 2 * qd : (2 * qd) & 3;
+  const int hc1 = G == 8 ? 2 * qd + 1 : (2 * qd + 1) & 3;
+
+  for (int i = slot; i < n_local; i += kSlots) {
+    const int st = i % NST;
+    // warp-uniform: a give-up on any lane ends the loop for the whole warp
+    if (!__all_sync(FULL, mbar_wait_bounded(&full[st], (i / NST) & 1, pool.status))) break;
+    const int ntok = flags[st];
+    if (ntok > 0) {
+      const uint32_t kb = sbase + st * STAGE;
+      if (ntok < kT) {
+        // a sequence's last block: zero the V rows past its last token (p = 0 there, and
+        // unwritten slots may hold any bits)
+        uint8_t* vst = smem + st * STAGE + CHUNK;
+        for (int x = lane; x < (kT - ntok) * (2 * D / 16); x += 32) {
+          const int r = ntok + x / (2 * D / 16), c = x % (2 * D / 16);
+          *reinterpret_cast<uint4*>(vst + (c >> 3) * kT * 128 + r * 128 + (c & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+      }
+      // ---- S = Q . K^T for tokens 0..7 (nt = 0) and 8..15 (nt = 1)
+      float sacc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+#pragma unroll
+        for (int k2 = 0; k2 < KS / 2; ++k2) {
+          uint32_t r0, r1, r2, r3;
+          ldsm_x4(kb + (k2 >> 1) * kT * 128 + nt * 1024 + krow + ((k2 & 1) ? kx1 : kx0), r0, r1, r2, r3);
+          mma_bf16_16816(sacc[nt], qa[2 * k2], r0, r1);
+          mma_bf16_16816(sacc[nt], qa[2 * k2 + 1], r2, r3);
+        }
+      }
+      // tokens 2qd, 2qd+1, 8+2qd, 9+2qd of head grp: hi row + lo row
+      float sc[4] = {sacc[0][0] + sacc[0][2], sacc[0][1] + sacc[0][3], sacc[1][0] + sacc[1][2],
+                     sacc[1][1] + sacc[1][3]};
+      if (ntok < kT) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if ((e >> 1) * 8 + 2 * qd + (e & 1) >= ntok) sc[e] = -INFINITY;
+      }
+      float bm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+      bm = fmaxf(bm, __shfl_xor_sync(FULL, bm, 1));
+      bm = fmaxf(bm, __shfl_xor_sync(FULL, bm, 2));
+      const float m_new = fmaxf(m_run, bm);
+      // rescale only when some head's running max grew (multiplying by 1 is exact)
+      if (__any_sync(FULL, m_new > m_run)) {
+        const float alpha = m_new > m_run ? fast_exp2(m_run - m_new) : 1.f;
+        l_run *= alpha;
+        const float a0 = __shfl_sync(FULL, alpha, hc0 * 4), a1 = __shfl_sync(FULL, alpha, hc1 * 4);
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+          for (int nt = 0; nt < NTP; ++nt) {
+            o[mt][nt][0] *= a0;
+            o[mt][nt][1] *= a1;
+            o[mt][nt][2] *= a0;
+            o[mt][nt][3] *= a1;
+          }
+      }
+      m_run = m_new;
+      const float mu = m_new == -INFINITY ? 0.f : m_new;
+      float pr[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) pr[e] = fast_exp2(sc[e] - mu);
+      l_run += (pr[0] + pr[1]) + (pr[2] + pr[3]);
+      uint32_t ph0, pl0, ph1, pl1;
+      split_bf16x2(pr[0], pr[1], ph0, pl0);  // tokens 2qd, 2qd+1   (B rows 0..7)
+      split_bf16x2(pr[2], pr[3], ph1, pl1);  // tokens 2qd+8, 2qd+9 (B rows 8..15)
+      uint32_t b0 = ph0, b1 = ph1;
+      if constexpr (G < 8) {
+        const uint32_t x0 = __shfl_xor_sync(FULL, pl0, 16), x1 = __shfl_xor_sync(FULL, pl1, 16);
+        if (grp >= 4) {
+          b0 = x0;
+          b1 = x1;
+        }
+      }
+      // ---- O^T += V^T . P^T, 16 value dims per tile
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        uint32_t a[4];
+        ldsm_x4_t(kb + vrow + (mt >> 2) * kT * 128 + ((((2 * (mt & 3) + vb) ^ r7)) << 4), a[0], a[1], a[2], a[3]);
+        mma_bf16_16816(o[mt][0], a, b0, b1);
+        if constexpr (G == 8) mma_bf16_16816(o[mt][1], a, pl0, pl1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+  }
+
+  // ---- l of head grp over the four token lanes; O = hi columns + lo columns
+  l_run += __shfl_xor_sync(FULL, l_run, 1);
+  l_run += __shfl_xor_sync(FULL, l_run, 2);
+  named_bar_sync(1, NCW * 32);  // every slot is done reading the stage ring
+  float* macc = reinterpret_cast<float*>(smem);
+  float2* mml = reinterpret_cast<float2*>(smem + NCW * G * D * 4);
+#pragma unroll
+  for (int mt = 0; mt < KS; ++mt) {
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if constexpr (G == 8)
+        v[e] = o[mt][0][e] + o[mt][NTP - 1][e];
+      else
+        v[e] = o[mt][0][e] + __shfl_xor_sync(FULL, o[mt][0][e], 2);
+    }
+    if (G == 8 || qd < 2) {
+      const int h0 = 2 * qd, h1 = 2 * qd + 1;
+      const int dl = 16 * mt + grp, dh = dl + 8;
+      if (h0 < G) {
+        macc[(warp * G + h0) * D + dl] = v[0];
+        macc[(warp * G + h0) * D + dh] = v[2];
+      }
+      if (h1 < G) {
+        macc[(warp * G + h1) * D + dl] = v[1];
+        macc[(warp * G + h1) * D + dh] = v[3];
+      }
+    }
+  }
+  if (qd == 0 && grp < G) mml[warp * G + grp] = make_float2(m_run, l_run);
+  named_bar_sync(1, NCW * 32);
+  attn_merge_combine<D, G, 1>(p, smem, b, g, s, warp, lane);
 }
 
 // ----------------------------------------------------------------------- combine
@@ -535,13 +846,48 @@ static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
   return cuda_check(cudaGetLastError(), "attention launch");
 }
 
-// Kernel shape per (D, G) and variant (G = 4 only; other G have one shape):
-//   0 automatic = 1: q in registers, 8-stage ring, three CTAs per SM
-//   2: 12-stage ring, two CTAs per SM        3: two warps per block (G/2 heads each)
-//   5: q in shared memory, 8-stage ring, three CTAs per SM
-// (Rings must be a multiple of the four consumer slots; see AttnCfg.)
+template <int D, int G, int NST, int MINB>
+static int launch_attn_mma(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
+  constexpr int smem = 1024 + (NST * 2 * kT * D * 2 + NST * 4 + 7) / 8 * 8 + 2 * NST * 8;
+  auto* fn = attn_mma_kernel<D, G, NST, MINB>;
+  // the HBM tier as a [rows][D] bf16 array, boxes of [T rows][64 dims], 128-byte swizzle
+  CUtensorMap tmap;
+  memset(&tmap, 0, sizeof(tmap));
+  const PoolView& v = p.pool;
+  if (v.blocks[0] > 0) {
+    const uint64_t rows = (uint64_t)v.blocks[0] * v.L * 2 * v.Hkv * v.T;
+    if (rows > (uint64_t)INT32_MAX) return set_error(DKV_ERR_UNSUPPORTED, "attention: HBM tier too large for TMA rows");
+    int rc = encode_bf16_2d(&tmap, v.tier[0], rows, (uint64_t)D, (uint32_t)kT);
+    if (rc) return rc;
+  }
+  static bool attr_done = false;  // per instantiation
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_check(e, "attention: set smem attribute");
+    attr_done = true;
+  }
+  dim3 grid(p.S, Hkv, B);
+  fn<<<grid, (kSlots + 1) * 32, smem, st>>>(p, tmap);
+  return cuda_check(cudaGetLastError(), "attention launch");
+}
+
+// Kernel per (D, G) and variant:
+//   0 automatic = 6: tensor cores, 8-stage ring, three CTAs per SM (G = 8: 12 stages, two)
+//   1: CUDA cores, q in registers, 8-stage ring, three CTAs per SM
+//   2: CUDA cores, 12-stage ring, two CTAs per SM   3: CUDA cores, two warps per block
+//   5: CUDA cores, q in shared memory
+// (2, 3, 5 exist for G = 4 only. Rings must be a multiple of the four consumer slots.)
 template <int D>
 static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant, cudaStream_t st) {
+  if (variant == 0 || variant == 6) {
+    switch (G) {
+      case 1: return launch_attn_mma<D, 1, 8, 3>(p, B, Hkv, st);
+      case 2: return launch_attn_mma<D, 2, 8, 3>(p, B, Hkv, st);
+      case 4: return launch_attn_mma<D, 4, 8, 3>(p, B, Hkv, st);
+      case 8: return launch_attn_mma<D, 8, 12, 2>(p, B, Hkv, st);
+    }
+    return set_error(DKV_ERR_UNSUPPORTED, "attention: unsupported G=%d", G);
+  }
   switch (G) {
     case 1: return launch_attn_t<D, 1, 1, 8, 3>(p, B, Hkv, st);
     case 2: return launch_attn_t<D, 2, 1, 8, 3>(p, B, Hkv, st);
@@ -559,7 +905,7 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
 }
 
 int attention_ctas_per_sm(int G, int variant) {
-  (void)G;
+  if (variant == 0 || variant == 6) return G == 8 ? 2 : 3;
   return variant == 2 || variant == 3 ? 2 : 3;
 }
 

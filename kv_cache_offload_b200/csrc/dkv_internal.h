@@ -1,6 +1,7 @@
 // Host-side internals shared by the libdkv translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stddef.h>
@@ -95,6 +96,9 @@ struct ProjArgs {
 };
 
 int launch_projection(const ProjArgs& a, cudaStream_t st);
+
+// 2-D bf16 tensor map over a row-major [rows][cols] array, box [box_rows][64], 128B swizzle.
+int encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // Workspace carve-up of one decode step (all offsets 256-byte aligned).
 struct DecodeWs {

@@ -202,7 +202,7 @@ def test_staged_calls_match_fused_step():
         ctx.close()
 
 
-@pytest.mark.parametrize("variant", [1, 2, 3, 5])  # 0 (automatic) is 1
+@pytest.mark.parametrize("variant", [1, 2, 3, 5, 6])  # 0 (automatic) is 6
 @pytest.mark.parametrize("splits", [1, 0])  # one split: long CTAs that wrap the stage ring
 @pytest.mark.parametrize("D", [64, 128])
 def test_attention_kernel_variants(variant, splits, D):
@@ -222,5 +222,33 @@ def test_attention_kernel_variants(variant, splits, D):
         TL.assert_out_close(out, TL.oracle_step(inp, layer=1)["out"], "variant %d" % variant)
         # same splits, same reduction order per (slot, head): the variants agree closely
         assert (out.float() - base.float()).abs().max().item() <= 2 ** -6
+    finally:
+        ctx.close()
+
+
+@pytest.mark.parametrize("D,Hq", [(128, 8), (64, 16)])
+def test_unwritten_tail_slots_are_ignored(D, Hq):
+    """Slots past a sequence's last cached token may hold any bits (here NaN in both tiers):
+    the outputs must not see them."""
+    cfg = WL.small_config(B=4, Hq=Hq, Hkv=2, D=D, H=256, ctx_range=(33, 300), host_prob=0.5)
+    inp = WL.make_decode_inputs(cfg, seed=23)
+    lay, T = inp.layout, cfg.T
+    tiers = [inp.hbm.view(torch.int16), inp.host.view(torch.int16)]
+    for b in range(cfg.B):
+        c = lay.seq_lens[b]
+        for pos in range(c + 1, (c // T + 1) * T):   # after the new token's slot
+            j, slot = divmod(pos, T)
+            t, phys = int(lay.tier_map[b, j]), int(lay.block_table[b, j])
+            tiers[t][0, phys, :, :, slot, :] = 0x7FC0   # bf16 quiet NaN
+        j = (c - 1) // T                                 # and the cached tail's own spare slots
+        t, phys = int(lay.tier_map[b, j]), int(lay.block_table[b, j])
+        for slot in range(c - j * T, T):
+            if j * T + slot != c:
+                tiers[t][0, phys, :, :, slot, :] = 0x7FC0
+    ctx = TL.make_pool(inp)
+    try:
+        out = TL.run_step(ctx, layer=0)
+        assert torch.isfinite(out.float()).all()
+        TL.assert_out_close(out, TL.oracle_step(inp, layer=0)["out"], "NaN in unwritten slots")
     finally:
         ctx.close()
