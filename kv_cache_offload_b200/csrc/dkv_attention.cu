@@ -872,18 +872,28 @@ static int launch_attn_mma(const AttnParams& p, int B, int Hkv, cudaStream_t st)
 }
 
 // Kernel per (D, G) and variant:
-//   0 automatic = 6: tensor cores, 8-stage ring, three CTAs per SM (G = 8: 12 stages, two)
+//   0 automatic = 6: tensor cores, 4-stage ring (one stage per consumer slot), four CTAs
+//     per SM (G = 8: 12 stages, two CTAs per SM); measured best on B200 for the 8B-shaped
+//     HBM layer (more resident CTAs beat deeper rings: 6.55 vs 6.16 TB/s)
+//   7: tensor cores, 8-stage ring, three CTAs per SM (G <= 4)
 //   1: CUDA cores, q in registers, 8-stage ring, three CTAs per SM
 //   2: CUDA cores, 12-stage ring, two CTAs per SM   3: CUDA cores, two warps per block
 //   5: CUDA cores, q in shared memory
 // (2, 3, 5 exist for G = 4 only. Rings must be a multiple of the four consumer slots.)
 template <int D>
 static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant, cudaStream_t st) {
-  if (variant == 0 || variant == 6) {
+  if (variant == 7 && G <= 4) {
     switch (G) {
       case 1: return launch_attn_mma<D, 1, 8, 3>(p, B, Hkv, st);
       case 2: return launch_attn_mma<D, 2, 8, 3>(p, B, Hkv, st);
       case 4: return launch_attn_mma<D, 4, 8, 3>(p, B, Hkv, st);
+    }
+  }
+  if (variant == 0 || variant == 6 || variant == 7) {
+    switch (G) {
+      case 1: return launch_attn_mma<D, 1, 4, 4>(p, B, Hkv, st);
+      case 2: return launch_attn_mma<D, 2, 4, 4>(p, B, Hkv, st);
+      case 4: return launch_attn_mma<D, 4, 4, 4>(p, B, Hkv, st);
       case 8: return launch_attn_mma<D, 8, 12, 2>(p, B, Hkv, st);
     }
     return set_error(DKV_ERR_UNSUPPORTED, "attention: unsupported G=%d", G);
@@ -905,7 +915,8 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
 }
 
 int attention_ctas_per_sm(int G, int variant) {
-  if (variant == 0 || variant == 6) return G == 8 ? 2 : 3;
+  if (variant == 0 || variant == 6) return G == 8 ? 2 : 4;
+  if (variant == 7) return G == 8 ? 2 : 3;
   return variant == 2 || variant == 3 ? 2 : 3;
 }
 
