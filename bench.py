@@ -84,7 +84,7 @@ def profiled_traffic(config_name: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(config_name)
-    if not e or e.get("src_hash") != src_hash("dkv_attention.cu", "dkv_common.cuh"):
+    if not e or e.get("src_hash") != src_hash("dkv_attention.cu", "dkv_common.cuh", "dkv_umma.cuh"):
         return None
     return e.get("bytes_per_launch")
 
@@ -807,13 +807,13 @@ def main():
                    "l2": "inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)},
         "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
         "stage_ms": {"project": stage_ms[0], "attend_and_combine": stage_ms[1]},
-        "roofline": ({"bound": "hbm", "kernel": "attn_splitk_kernel",
+        "roofline": ({"bound": "hbm", "kernel": "attn_mma_kernel",
                       "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                       "peak_source": peak_kind,
                       "traffic": profiled_traffic(cfg.name),
                       "algorithmic_bytes_per_launch": wl.kv_bytes}
                      if not wl.kv_host_bytes else
-                     {"bound": "host_link", "kernel": "attn_splitk_kernel",
+                     {"bound": "host_link", "kernel": "attn_mma_kernel",
                       "achieved": host_info["achieved_gbs"], "peak": host_info["h2d_peak_gbs"], "unit": "GB/s",
                       "frac": host_info["frac"], "peak_source": "measured cudaMemcpy H2D (pinned, 1 GiB) in this run",
                       "traffic": None, "algorithmic_bytes_per_launch": wl.kv_host_bytes}),
