@@ -32,6 +32,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <utility>
+
 #include "dkv_internal.h"
 #include "dkv_umma.cuh"
 
@@ -307,6 +309,9 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const PoolView& pool = p.pool;
+  // everything read below (tables, q, counters) comes from the kernels ahead in the stream
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   // cached tokens of this sequence, clamped to what the table can hold
   int ctx = p.seq_lens[b];
@@ -617,6 +622,9 @@ __global__ void __launch_bounds__((kSlots + 1) * 32, MINB)
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const PoolView& pool = p.pool;
+  // everything read below (tables, q, counters) comes from the kernels ahead in the stream
+  griddep_wait();
+  if (threadIdx.x == 0) griddep_launch_dependents();
 
   int ctx = p.seq_lens[b];
   if (ctx < 0 || ctx / kT + 1 > p.max_blocks) {
@@ -830,6 +838,23 @@ __global__ void __launch_bounds__(D) combine_kernel(int Hq, int Hkv, int S,
 
 // ---------------------------------------------------------------------- launchers
 
+// Launch with programmatic stream serialization: the kernel may be scheduled while the
+// projection ahead of it finishes; it waits for it (griddep_wait) before reading anything.
+template <typename... KArgs, typename... Args>
+static int launch_pdl(void (*fn)(KArgs...), dim3 grid, int threads, int smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1] = {};
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cuda_check(cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...), "attention launch");
+}
+
 template <int D, int HPW, int WPB, int NST, int MINB, bool QS = false>
 static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
   using C = AttnCfg<D, HPW, WPB, NST>;
@@ -841,9 +866,7 @@ static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
     if (e != cudaSuccess) return cuda_check(e, "attention: set smem attribute");
     attr_done = true;
   }
-  dim3 grid(p.S, Hkv, B);
-  fn<<<grid, C::THREADS, smem, st>>>(p);
-  return cuda_check(cudaGetLastError(), "attention launch");
+  return launch_pdl(fn, dim3(p.S, Hkv, B), C::THREADS, smem, st, p);
 }
 
 template <int D, int G, int NST, int MINB>
@@ -866,9 +889,7 @@ static int launch_attn_mma(const AttnParams& p, int B, int Hkv, cudaStream_t st)
     if (e != cudaSuccess) return cuda_check(e, "attention: set smem attribute");
     attr_done = true;
   }
-  dim3 grid(p.S, Hkv, B);
-  fn<<<grid, (kSlots + 1) * 32, smem, st>>>(p, tmap);
-  return cuda_check(cudaGetLastError(), "attention launch");
+  return launch_pdl(fn, dim3(p.S, Hkv, B), (kSlots + 1) * 32, smem, st, p, tmap);
 }
 
 // Kernel per (D, G) and variant:

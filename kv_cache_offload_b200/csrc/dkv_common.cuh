@@ -52,6 +52,17 @@ __device__ __forceinline__ void flag_error(int* status, int bits) {
   if (status) atomicOr(status, bits);
 }
 
+// ---------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before the kernel
+// ahead of it in the stream has finished. griddep_wait() blocks the calling thread until
+// that kernel has completed and its memory is visible (a no-op for a normal launch);
+// griddep_launch_dependents() lets the next such kernel start once every CTA of this grid
+// has signalled (or exited). Both exist on sm_90 and later.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ shared memory
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

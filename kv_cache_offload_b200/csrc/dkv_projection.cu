@@ -120,7 +120,19 @@ __global__ void __launch_bounds__(kPThreads, 2)
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
-    for (int s = 0; s < nsteps; ++s) {
+    // The first ring's W tiles do not depend on the kernel ahead in the stream (weights are
+    // never written by it), so they are fetched before waiting for it; x and everything
+    // after come once it has completed.
+    const int pre = nsteps < nst ? nsteps : nst;
+    for (int s = 0; s < pre; ++s) {
+      uint8_t* wdst = smem + s * stage_bytes;
+      mbar_arrive_expect_tx(&full[s], (uint32_t)(np * p.D * 128 + xtile));
+      for (int i = 0; i < np; ++i)
+        tma_load_2d(wdst + i * p.D * 128, &tmW, (kb0 + s) * 64, piece_row(p, g, t * p.ppt + i), &full[s]);
+    }
+    griddep_wait();
+    for (int s = 0; s < pre; ++s) tma_load_2d(smem + s * stage_bytes + kWTile, &tmX, (kb0 + s) * 64, 0, &full[s]);
+    for (int s = pre; s < nsteps; ++s) {
       const int st = s % nst, n = s / nst;
       if (n > 0 && !mbar_wait_bounded(&empty[st], (n - 1) & 1, p.pool.status)) break;
       const int kb = kb0 + s;
@@ -146,8 +158,13 @@ __global__ void __launch_bounds__(kPThreads, 2)
       umma_commit(&empty[st]);
     }
     umma_commit(done);
+  } else {
+    // the tables, positions and workspace below belong to the kernels ahead in the stream
+    griddep_wait();
+    if (tid == 64) griddep_launch_dependents();
   }
   __syncwarp();
+  griddep_wait();
 
   // ----------------------------------------------------- TMEM -> shared partial [n][row]
   mbar_wait_bounded(done, 0, p.pool.status);
@@ -302,17 +319,19 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
   if (CS > 8) CS = 8;
   if (CS > p.KB) CS = p.KB;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute at[1] = {};
+  cudaLaunchAttribute at[2] = {};
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = CS;
   at[0].val.clusterDim.y = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   at[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(CS, tiles, 1);
   cfg.blockDim = dim3(kPThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   p.CS = CS;
   cudaError_t e = cudaLaunchKernelEx(&cfg, proj_umma_kernel, tmW, tmX, p);
   return cuda_check(e, "projection launch");
