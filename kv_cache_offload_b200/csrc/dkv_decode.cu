@@ -15,14 +15,24 @@ namespace dkv {
 
 // ----------------------------------------------------------------- workspace
 
-// Automatic split count: about 2.9 waves of resident CTAs (measured best on B200 for the
-// HBM-resident 8B-shaped layer; host-bound configurations are insensitive to it).
+// Automatic split count. Tensor-core kernels: one wave of about 7/8 of the resident CTA
+// slots, at most 32 splits (the last split CTA of each (sequence, kv head) merges all of
+// them). Measured best on B200 for uniform batches of 2 K - 32 K tokens, B = 4..32 (8B
+// shape, B=16 x 32 K: 311 us at 4 splits vs 326 us at 13 = 2.8 waves); more waves only
+// add per-CTA setup and merge work. CUDA-core kernels: about 2.9 waves (their best).
+// Host-bound configurations are insensitive to the split count.
 static int pick_attn_splits(const dkv_pool* pool, int B, int Hkv, int G, int max_blocks) {
   int s = pool->tuning.attn_splits;
   if (s <= 0) {
-    const int slots = pool->num_sms * attention_ctas_per_sm(G, pool->tuning.attn_variant);
+    const int variant = pool->tuning.attn_variant;
+    const int slots = pool->num_sms * attention_ctas_per_sm(G, variant);
     const int units = B * Hkv;
-    s = (29 * slots + 5 * units) / (10 * units);
+    if (variant == 0 || variant == 6 || variant == 7) {
+      s = (7 * slots + 4 * units) / (8 * units);  // round(7/8 * slots / units)
+      if (s > 32) s = 32;
+    } else {
+      s = (29 * slots + 5 * units) / (10 * units);
+    }
   }
   if (s > max_blocks) s = max_blocks;
   return s < 1 ? 1 : s;
