@@ -86,7 +86,10 @@ typedef struct dkv_tuning {
                             for G = 4 also 2 (CUDA cores, 12-stage ring), 3 (two warps
                             per block), 5 (q in shared memory); 4 is invalid */
   int32_t attn_lsu_hbm;  /* 1: load HBM-tier blocks with 16-byte cp.async, not bulk copies */
-  int32_t reserved[4];
+  int32_t serial_launch; /* 1: launch the decode kernels without programmatic dependent
+                            launch (each starts when the one before has finished; for
+                            timing the kernels one by one); 0: overlap their boundaries */
+  int32_t reserved[3];
 } dkv_tuning;
 
 /*

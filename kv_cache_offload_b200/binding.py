@@ -58,7 +58,7 @@ class dkv_pool_config(ctypes.Structure):
 class dkv_tuning(ctypes.Structure):
     _fields_ = [("attn_splits", ctypes.c_int32), ("proj_splits", ctypes.c_int32),
                 ("attn_variant", ctypes.c_int32), ("attn_lsu_hbm", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 4)]
+                ("serial_launch", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
 
 
 class dkv_bm_config(ctypes.Structure):
@@ -216,8 +216,8 @@ def dkv_pool_tier_ptr(pool: int, tier: int):
 
 
 def dkv_pool_set_tuning(pool: int, attn_splits: int = 0, proj_splits: int = 0,
-                        attn_variant: int = 0, attn_lsu_hbm: int = 0):
-    t = dkv_tuning(attn_splits, proj_splits, attn_variant, attn_lsu_hbm)
+                        attn_variant: int = 0, attn_lsu_hbm: int = 0, serial_launch: int = 0):
+    t = dkv_tuning(attn_splits, proj_splits, attn_variant, attn_lsu_hbm, serial_launch)
     _chk(lib().dkv_pool_set_tuning(pool, ctypes.byref(t)))
 
 

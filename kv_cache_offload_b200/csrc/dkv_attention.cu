@@ -221,8 +221,8 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
     if ((i & 31) == 0) {
       const int j = j0 + i + lane;
       if (j < j1) {
-        pf_tier = p.tier_map[rowbase + j];
-        pf_phys = p.table[rowbase + j];
+        pf_tier = __ldcg(p.tier_map + rowbase + j);  // L2: tables may be rewritten between launches
+        pf_phys = __ldcg(p.table + rowbase + j);
       }
     }
     const int st = i % NST;
@@ -622,11 +622,15 @@ __global__ void __launch_bounds__((kSlots + 1) * 32, MINB)
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const PoolView& pool = p.pool;
-  // everything read below (tables, q, counters) comes from the kernels ahead in the stream
-  griddep_wait();
+  // Launched with programmatic dependent launch behind the projection: q, the new token's
+  // k/v and the split counters come from it, so the consumers wait for it (griddep_wait)
+  // before touching them. The tables, the positions and the cached blocks were finished
+  // by the kernels before it (the projection signals only after its own wait), and the
+  // one cache slot it writes is masked here, so the producer starts at once. Tables and
+  // positions are read through L2.
   if (threadIdx.x == 0) griddep_launch_dependents();
 
-  int ctx = p.seq_lens[b];
+  int ctx = __ldcg(p.seq_lens + b);
   if (ctx < 0 || ctx / kT + 1 > p.max_blocks) {
     if (threadIdx.x == 0 && s == 0 && g == 0) flag_error(pool.status, kErrCtxTooLong);
     ctx = ctx < 0 ? 0 : min(ctx, p.max_blocks * kT);
@@ -654,6 +658,7 @@ __global__ void __launch_bounds__((kSlots + 1) * 32, MINB)
   const int slot = warp;
   const int grp = lane >> 2, qd = lane & 3;
   constexpr unsigned FULL = 0xffffffffu;
+  griddep_wait();  // q, k_hat, v_hat and the counters are the projection's
 
   // q of head grp as A fragments: rows grp (hi) and grp + 8 (lo), dims 16ks + 2qd + {0,1,8,9}
   uint32_t qa[KS][4];
@@ -841,7 +846,8 @@ __global__ void __launch_bounds__(D) combine_kernel(int Hq, int Hkv, int S,
 // Launch with programmatic stream serialization: the kernel may be scheduled while the
 // projection ahead of it finishes; it waits for it (griddep_wait) before reading anything.
 template <typename... KArgs, typename... Args>
-static int launch_pdl(void (*fn)(KArgs...), dim3 grid, int threads, int smem, cudaStream_t st, Args&&... args) {
+static int launch_pdl(void (*fn)(KArgs...), dim3 grid, int threads, int smem, cudaStream_t st, bool pdl,
+                      Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[1] = {};
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -851,7 +857,7 @@ static int launch_pdl(void (*fn)(KArgs...), dim3 grid, int threads, int smem, cu
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 1 : 0;
   return cuda_check(cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...), "attention launch");
 }
 
@@ -866,7 +872,7 @@ static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
     if (e != cudaSuccess) return cuda_check(e, "attention: set smem attribute");
     attr_done = true;
   }
-  return launch_pdl(fn, dim3(p.S, Hkv, B), C::THREADS, smem, st, p);
+  return launch_pdl(fn, dim3(p.S, Hkv, B), C::THREADS, smem, st, p.pdl != 0, p);
 }
 
 template <int D, int G, int NST, int MINB>
@@ -889,7 +895,7 @@ static int launch_attn_mma(const AttnParams& p, int B, int Hkv, cudaStream_t st)
     if (e != cudaSuccess) return cuda_check(e, "attention: set smem attribute");
     attr_done = true;
   }
-  return launch_pdl(fn, dim3(p.S, Hkv, B), (kSlots + 1) * 32, smem, st, p, tmap);
+  return launch_pdl(fn, dim3(p.S, Hkv, B), (kSlots + 1) * 32, smem, st, p.pdl != 0, p, tmap);
 }
 
 // Kernel per (D, G) and variant:

@@ -123,6 +123,7 @@ int dkv_decode_project(dkv_pool* pool, int layer, const uint16_t* x, const uint1
   a.vnew = reinterpret_cast<float*>(ws + w.off_vnew);
   a.attn_cnt = reinterpret_cast<int*>(ws + w.off_cnt);
   a.cluster = pool->tuning.proj_splits;
+  a.pdl = !pool->tuning.serial_launch;
   return launch_projection(a, (cudaStream_t)stream);
 }
 
@@ -153,6 +154,7 @@ int dkv_decode_attend(dkv_pool* pool, int layer, const int32_t* block_table, con
   a.vnew = reinterpret_cast<const float*>(ws + w.off_vnew);
   a.out = out;
   a.lsu_hbm = pool->tuning.attn_lsu_hbm;
+  a.pdl = !pool->tuning.serial_launch;
   return launch_attention(a, B, w.Hkv, w.D, w.G, pool->tuning.attn_variant, (cudaStream_t)stream);
 }
 

@@ -68,6 +68,7 @@ struct AttnParams {
   const float* vnew; // [B][Hkv][D]
   uint16_t* out;     // [B][Hq*D] bf16, or nullptr
   int lsu_hbm;       // load HBM-tier blocks with cp.async instead of bulk copies
+  int pdl;           // launch with programmatic dependent launch
 };
 
 int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, int variant, cudaStream_t st);
@@ -93,6 +94,7 @@ struct ProjArgs {
   float* vnew;    // [B][Hkv][D]  v_hat as fp32
   int* attn_cnt;  // [B][Hkv] attention split counters, reset by the projection
   int cluster;    // cluster size request (0 = automatic)
+  int pdl;        // launch with programmatic dependent launch
 };
 
 int launch_projection(const ProjArgs& a, cudaStream_t st);

@@ -331,7 +331,7 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cfg.attrs = at;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = a.pdl ? 2 : 1;
   p.CS = CS;
   cudaError_t e = cudaLaunchKernelEx(&cfg, proj_umma_kernel, tmW, tmX, p);
   return cuda_check(e, "projection launch");

@@ -252,3 +252,26 @@ def test_unwritten_tail_slots_are_ignored(D, Hq):
         TL.assert_out_close(out, TL.oracle_step(inp, layer=0)["out"], "NaN in unwritten slots")
     finally:
         ctx.close()
+
+
+def test_serial_launch_matches_overlapped_launch():
+    """Programmatic dependent launch only moves kernel starts: outputs are bit-identical
+    with the kernels launched one after another."""
+    cfg = WL.small_config(B=5, Hq=16, Hkv=2, D=128, H=512, ctx_range=(100, 900), host_prob=0.3)
+    inp = WL.make_decode_inputs(cfg, seed=31)
+    ctx = TL.make_pool(inp)
+    try:
+        a = TL.run_step(ctx, layer=1)
+        dkv.dkv_pool_set_tuning(ctx.pool, serial_launch=1)
+        x, W = inp.x.cuda(), inp.W.cuda()
+        b = torch.empty_like(a)
+        nws = dkv.dkv_decode_workspace_bytes(ctx.pool, cfg.B, ctx.table.shape[1], cfg.Hq, cfg.H)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        for _ in range(3):  # back to back on one stream, as a serving loop runs them
+            dkv.dkv_decode_step(ctx.pool, 1, x, W, ctx.table, ctx.seq_lens, ctx.tier_map, cfg.Hq, cfg.theta, b, ws)
+        assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+        with pytest.raises(dkv.DkvError):
+            dkv.dkv_pool_set_tuning(ctx.pool, serial_launch=2)
+    finally:
+        ctx.close()
