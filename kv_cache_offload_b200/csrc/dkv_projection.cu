@@ -67,6 +67,13 @@ __device__ __forceinline__ float dsmem_ld(uint32_t addr) {
   return v;
 }
 
+// Epilogue lookups done while W streams, for the first four sequences a CTA finishes:
+// the position and the two cache-slot addresses (key, value) of kv head g.
+struct EpiPre {
+  int pos[4];
+  uint16_t* dst[4][2];
+};
+
 // First W row of piece (head) `pc` of kv-head group g: pieces 0..G-1 are the group's q
 // heads, G its key head, G+1 its value head.
 __device__ __forceinline__ int piece_row(const ProjParams& p, int g, int pc) {
@@ -97,6 +104,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   float* rowx = reinterpret_cast<float*>(smem + nst * stage_bytes + 256);  // [128]
   float* part = reinterpret_cast<float*>(smem);  // [Npad][128], aliases the ring later
+  EpiPre* pre = reinterpret_cast<EpiPre*>(smem + nst * stage_bytes + 128);  // after the barriers
 
   if (tid == 0) {
     for (int i = 0; i < nst; ++i) {
@@ -162,6 +170,35 @@ __global__ void __launch_bounds__(kPThreads, 2)
     // the tables, positions and workspace below belong to the kernels ahead in the stream
     griddep_wait();
     if (tid == 64) griddep_launch_dependents();
+    if (tid >= 64 && tid < 68) {
+      // while W streams: position and cache-slot addresses of sequence rank + CS * i
+      const int i = tid - 64, b = rank + p.CS * i;
+      int pos = 0;
+      uint16_t* dk = nullptr;
+      uint16_t* dv = nullptr;
+      if (b < p.B) {
+        pos = p.seq_lens[b];
+        const int64_t jb = pos >= 0 ? (int64_t)pos / p.pool.T : -1;
+        if (jb < 0 || jb >= p.max_blocks) {
+          flag_error(p.pool.status, kErrCtxTooLong);
+        } else {
+          const int tier = p.tier_map[(int64_t)b * p.max_blocks + jb];
+          const int64_t phys = p.table[(int64_t)b * p.max_blocks + jb];
+          if (tier > 1) {
+            flag_error(p.pool.status, kErrBadTier);
+          } else if (phys < 0 || phys >= tier_blocks(p.pool, tier)) {
+            flag_error(p.pool.status, kErrBadBlock);
+          } else {
+            const int64_t slot = (int64_t)(pos % p.pool.T) * p.D;
+            dk = tier_base(p.pool, tier) + chunk_offset(p.pool, tier, p.layer, phys, 0, g) + slot;
+            dv = tier_base(p.pool, tier) + chunk_offset(p.pool, tier, p.layer, phys, 1, g) + slot;
+          }
+        }
+      }
+      pre->pos[i] = pos;
+      pre->dst[i][0] = dk;
+      pre->dst[i][1] = dv;
+    }
   }
   __syncwarp();
   griddep_wait();
@@ -189,7 +226,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
   uint32_t rbase[16];
 #pragma unroll
   for (int q = 0; q < 16; ++q) rbase[q] = dsmem_map(part, q < p.CS ? q : 0);
-  for (int b = rank; b < p.B; b += p.CS) {
+  for (int b = rank, it = 0; b < p.B; b += p.CS, ++it) {
     const uint32_t off = (uint32_t)((b * 128 + row) * 4);
     float vals[16];
 #pragma unroll
@@ -202,7 +239,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
     const float xp = rowx[partner];
     __syncthreads();
     if (!live) continue;
-    const int pos = p.seq_lens[b];
+    const int pos = it < 4 ? pre->pos[it] : p.seq_lens[b];
     if (pc <= p.G) {
       // rotate-half RoPE: angle reduced mod 2*pi in fp64, then a single-precision sincos
       const double ang = (double)pos * p.inv_freq[pi];
@@ -219,7 +256,12 @@ __global__ void __launch_bounds__(kPThreads, 2)
     const uint16_t hb = f32_to_bf16_bits(x);
     const int kv = pc == p.G ? 0 : 1;
     (kv ? p.vnew : p.knew)[((int64_t)b * p.Hkv + g) * D + d] = __uint_as_float((uint32_t)hb << 16);
-    // the single cache write: slot pos mod T of logical block pos / T
+    // the single cache write: slot pos mod T of logical block pos / T (looked up while W
+    // streamed for the first four sequences; bad entries were flagged there)
+    if (it < 4) {
+      if (pre->dst[it][kv]) pre->dst[it][kv][d] = hb;
+      continue;
+    }
     const int64_t jb = pos >= 0 ? (int64_t)pos / p.pool.T : -1;
     if (jb < 0 || jb >= p.max_blocks) {
       flag_error(p.pool.status, kErrCtxTooLong);

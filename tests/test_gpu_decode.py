@@ -275,3 +275,28 @@ def test_serial_launch_matches_overlapped_launch():
             dkv.dkv_pool_set_tuning(ctx.pool, serial_launch=2)
     finally:
         ctx.close()
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_empty_context_returns_the_new_value_exactly(layout):
+    """With no cached tokens the softmax has one term: every q head of a group outputs the
+    new value v_hat of its kv head, bit for bit (the value the step wrote into the cache)."""
+    cfg = WL.small_config(B=4, Hq=8, Hkv=2, D=128, H=256, host_prob=0.5)
+    inp = WL.make_decode_inputs(cfg, seed=41, pool_layout=layout, seq_lens=[0, 37, 0, 16])
+    ctx = TL.make_pool(inp)
+    try:
+        out = TL.run_step(ctx, layer=1).view(torch.int16).cpu().reshape(cfg.B, cfg.Hq, cfg.D)
+        torch.cuda.synchronize()
+        tiers = [ctx.hbm.cpu().view(torch.int16).reshape(inp.hbm.shape),
+                 ctx.host.clone().reshape(inp.host.shape)]
+        lay, G = inp.layout, cfg.Hq // cfg.Hkv
+        for b in (0, 2):
+            t, phys = int(lay.tier_map[b, 0]), int(lay.block_table[b, 0])
+            for h in range(cfg.Hq):
+                g = h // G
+                vhat = tiers[t][1, phys, 1, g, 0] if layout == 0 else tiers[t][phys, 1, 1, g, 0]
+                assert torch.equal(out[b, h], vhat), (b, h)
+        TL.assert_out_close(out.view(torch.bfloat16).reshape(cfg.B, -1).cuda(),
+                            TL.oracle_step(inp, layer=1)["out"], "empty contexts")
+    finally:
+        ctx.close()
