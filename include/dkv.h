@@ -87,8 +87,9 @@ typedef struct dkv_tuning {
                             per block), 5 (q in shared memory); 4 is invalid */
   int32_t attn_lsu_hbm;  /* 1: load HBM-tier blocks with 16-byte cp.async, not bulk copies */
   int32_t serial_launch; /* 1: launch the decode kernels without programmatic dependent
-                            launch (each starts when the one before has finished; for
-                            timing the kernels one by one); 0: overlap their boundaries */
+                            launch (each starts when the one before has finished: for
+                            timing the kernels one by one, or when Wqkv is written by the
+                            kernel directly ahead); 0: overlap their boundaries */
   int32_t reserved[3];
 } dkv_tuning;
 
@@ -165,8 +166,17 @@ size_t dkv_decode_workspace_bytes(const dkv_pool* pool, int B, int max_blocks,
  * out: device [B][Hq*D] bf16. workspace: device, >= dkv_decode_workspace_bytes(...),
  * 256-byte aligned; its contents need no initialisation.
  * Supported: 1 <= B <= 32, hidden % 64 == 0, Hq % Hkv == 0 with Hq/Hkv in {1,2,4,8}.
- * Two stream-ordered kernels (projection; attention with the split combine fused); no host
+ * Two kernels (projection; attention with the split combine fused); no host
  * synchronisation, no allocation, so the call can be captured into a CUDA graph.
+ * Unless serial_launch is set (dkv_tuning), they are launched with programmatic dependent
+ * launch: the projection may start while the kernel ahead of it in the stream is still
+ * running, if that kernel signals programmatic launch completion early (this library's
+ * kernels do), and then fetches part of Wqkv before waiting for it; everything else
+ * (x, tables, positions, workspace, cache) is touched only after that kernel has
+ * finished. So Wqkv must not be written by the kernel directly ahead of this call when
+ * that kernel signals early. The attention streams cached KV while the projection
+ * finishes (it writes only a slot the attention masks) and reads the projection's
+ * outputs after it has finished. Seen from the stream, the call is ordered as usual.
  */
 int dkv_decode_step(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t* Wqkv,
                     const int32_t* block_table, const int32_t* seq_lens,
@@ -184,6 +194,8 @@ int dkv_decode_step(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t
  *            partial states with the new token's term (score q . k_hat, value v_hat) into
  *            out (the combine, fused).
  *   combine: the merge as its own kernel, for attend(out = NULL).
+ * Called on its own, attend waits for the kernel ahead of it before reading anything
+ * (only inside dkv_decode_step does it stream cached KV while the projection finishes).
  */
 int dkv_decode_project(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t* Wqkv,
                        const int32_t* block_table, const int32_t* seq_lens,

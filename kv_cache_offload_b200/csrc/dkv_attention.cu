@@ -622,12 +622,14 @@ __global__ void __launch_bounds__((kSlots + 1) * 32, MINB)
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const PoolView& pool = p.pool;
-  // Launched with programmatic dependent launch behind the projection: q, the new token's
-  // k/v and the split counters come from it, so the consumers wait for it (griddep_wait)
-  // before touching them. The tables, the positions and the cached blocks were finished
-  // by the kernels before it (the projection signals only after its own wait), and the
-  // one cache slot it writes is masked here, so the producer starts at once. Tables and
-  // positions are read through L2.
+  // Launched with programmatic dependent launch behind the projection of the same step
+  // (p.early_kv): q, the new token's k/v and the split counters come from it, so the
+  // consumers wait for it (griddep_wait) before touching them. The tables, the positions
+  // and the cached blocks were finished by the kernels before it (the projection signals
+  // only after its own wait), and the one cache slot it writes is masked here, so the
+  // producer starts at once; tables and positions are read through L2. Launched behind
+  // anything else, every thread waits first.
+  if (!p.early_kv) griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
 
   int ctx = __ldcg(p.seq_lens + b);

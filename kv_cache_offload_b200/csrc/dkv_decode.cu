@@ -127,9 +127,11 @@ int dkv_decode_project(dkv_pool* pool, int layer, const uint16_t* x, const uint1
   return launch_projection(a, (cudaStream_t)stream);
 }
 
-int dkv_decode_attend(dkv_pool* pool, int layer, const int32_t* block_table, const int32_t* seq_lens,
-                      const uint8_t* tier_map, int B, int max_blocks, int hidden, int num_q_heads,
-                      uint16_t* out, void* workspace, size_t ws_bytes, void* stream) {
+namespace dkv {
+// early_kv: the kernel ahead in the stream is this step's projection (dkv_decode_step)
+static int decode_attend(dkv_pool* pool, int layer, const int32_t* block_table, const int32_t* seq_lens,
+                         const uint8_t* tier_map, int B, int max_blocks, int hidden, int num_q_heads,
+                         uint16_t* out, void* workspace, size_t ws_bytes, void* stream, bool early_kv) {
   if (!pool || !block_table || !seq_lens || !tier_map)
     return set_error(DKV_ERR_ARG, "dkv_decode_attend: null argument");
   DecodeWs w;
@@ -155,7 +157,16 @@ int dkv_decode_attend(dkv_pool* pool, int layer, const int32_t* block_table, con
   a.out = out;
   a.lsu_hbm = pool->tuning.attn_lsu_hbm;
   a.pdl = !pool->tuning.serial_launch;
+  a.early_kv = early_kv && a.pdl;
   return launch_attention(a, B, w.Hkv, w.D, w.G, pool->tuning.attn_variant, (cudaStream_t)stream);
+}
+}  // namespace dkv
+
+extern "C" int dkv_decode_attend(dkv_pool* pool, int layer, const int32_t* block_table, const int32_t* seq_lens,
+                                 const uint8_t* tier_map, int B, int max_blocks, int hidden, int num_q_heads,
+                                 uint16_t* out, void* workspace, size_t ws_bytes, void* stream) {
+  return decode_attend(pool, layer, block_table, seq_lens, tier_map, B, max_blocks, hidden, num_q_heads, out,
+                       workspace, ws_bytes, stream, false);
 }
 
 int dkv_decode_combine(dkv_pool* pool, int B, int max_blocks, int hidden, int num_q_heads, uint16_t* out,
@@ -180,8 +191,8 @@ int dkv_decode_step(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t
   int rc = dkv_decode_project(pool, layer, x, Wqkv, block_table, seq_lens, tier_map, B, max_blocks, hidden,
                               num_q_heads, rope_theta, workspace, ws_bytes, stream);
   if (rc) return rc;
-  return dkv_decode_attend(pool, layer, block_table, seq_lens, tier_map, B, max_blocks, hidden, num_q_heads,
-                           out, workspace, ws_bytes, stream);
+  return decode_attend(pool, layer, block_table, seq_lens, tier_map, B, max_blocks, hidden, num_q_heads, out,
+                       workspace, ws_bytes, stream, true);
 }
 
 }  // extern "C"

@@ -69,6 +69,7 @@ struct AttnParams {
   uint16_t* out;     // [B][Hq*D] bf16, or nullptr
   int lsu_hbm;       // load HBM-tier blocks with cp.async instead of bulk copies
   int pdl;           // launch with programmatic dependent launch
+  int early_kv;      // the kernel ahead is this step's projection: stream KV before it ends
 };
 
 int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, int variant, cudaStream_t st);
