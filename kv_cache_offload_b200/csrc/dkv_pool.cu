@@ -250,9 +250,9 @@ int dkv_pool_tier_ptr(const dkv_pool* p, int tier, void** dev_ptr, void** host_p
 int dkv_pool_set_tuning(dkv_pool* p, const dkv_tuning* t) {
   if (!p) return set_error(DKV_ERR_ARG, "dkv_pool_set_tuning: null pool");
   if (t) {
-    if (t->attn_splits < 0 || t->proj_splits < 0 || t->proj_splits > 16 || t->attn_variant < 0 ||
-        t->attn_variant > 7 || t->attn_variant == 4 || t->attn_lsu_hbm < 0 || t->attn_lsu_hbm > 1 ||
-        t->serial_launch < 0 || t->serial_launch > 1)
+    const int v = t->attn_variant;
+    if (t->attn_splits < 0 || t->proj_splits < 0 || t->proj_splits > 16 || (v != 0 && v != 1 && v != 6 && v != 7) ||
+        t->attn_lsu_hbm < 0 || t->attn_lsu_hbm > 1 || t->serial_launch < 0 || t->serial_launch > 1)
       return set_error(DKV_ERR_ARG, "dkv_pool_set_tuning: value out of range");
     p->tuning = *t;
   } else {
