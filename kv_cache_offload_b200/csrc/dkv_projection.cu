@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
   const int g = tile / p.nt, t = tile % p.nt;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // 1024-byte aligned carve-up: ring | barriers | tmem slot | row exchange
+  // 1024-byte aligned carve-up: ring | barriers | tmem slot | epilogue lookups
   const uint32_t base_u = smem_u32(psmem_raw);
   uint8_t* smem = psmem_raw + (((base_u + 1023u) & ~1023u) - base_u);
   const int xtile = p.Npad * 128;
@@ -102,7 +102,6 @@ __global__ void __launch_bounds__(kPThreads, 2)
   uint64_t* empty = full + nst;
   uint64_t* done = empty + nst;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  float* rowx = reinterpret_cast<float*>(smem + nst * stage_bytes + 256);  // [128]
   float* part = reinterpret_cast<float*>(smem);  // [Npad][128], aliases the ring later
   EpiPre* pre = reinterpret_cast<EpiPre*>(smem + nst * stage_bytes + 128);  // after the barriers
 
@@ -217,12 +216,14 @@ __global__ void __launch_bounds__(kPThreads, 2)
   cluster.sync();  // every CTA's partial is in its shared memory
 
   // ------------------------------------ column reduction over the cluster + epilogue
-  // thread = tile row: head row / D of the tile, dim d = row % D of that head
-  const int D = p.D, half = D / 2, row = tid;
+  // thread -> tile row (head row / D of the tile, dim d = row % D of that head), mapped so
+  // that the two rows of a RoPE pair (d and d + D/2) sit in lanes l and l ^ 16 of one
+  // warp: the pair exchange is a shuffle, with no block barrier per sequence
+  const int D = p.D, half = D / 2, wph = D / 32;  // warps per head
+  const int row = (warp / wph) * D + (warp % wph) * 16 + (lane & 15) + ((lane & 16) ? half : 0);
   const int pc = t * p.ppt + row / D;     // piece (head) index within the group
   const int d = row % D, pi = d % half;   // RoPE pair index
   const bool live = row / D < np;
-  const int partner = d < half ? row + half : row - half;
   uint32_t rbase[16];
 #pragma unroll
   for (int q = 0; q < 16; ++q) rbase[q] = dsmem_map(part, q < p.CS ? q : 0);
@@ -234,10 +235,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
     float x = 0.f;
 #pragma unroll
     for (int q = 0; q < 16; ++q) x += vals[q];  // rank order: deterministic
-    rowx[row] = x;
-    __syncthreads();
-    const float xp = rowx[partner];
-    __syncthreads();
+    const float xp = __shfl_xor_sync(0xffffffffu, x, 16);  // the pair's other row
     if (!live) continue;
     const int pos = it < 4 ? pre->pos[it] : p.seq_lens[b];
     if (pc <= p.G) {
@@ -313,7 +311,7 @@ int encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t col
 }
 
 static size_t proj_smem_bytes(int Npad, int nst) {
-  return 1024 + (size_t)nst * (kWTile + Npad * 128) + 256 + 128 * 4;
+  return 1024 + (size_t)nst * (kWTile + Npad * 128) + 256;
 }
 
 int launch_projection(const ProjArgs& a, cudaStream_t st) {
