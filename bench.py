@@ -326,6 +326,16 @@ def cpu_baseline(cfg, seed, budget_s):
 # --------------------------------------------------------------------------- main
 
 
+def workload_config(cfg: WL.DecodeConfig, world: int) -> dict:
+    """The `config` object both arms report for a decode workload."""
+    seq_len = cfg.ctx or cfg.ctx_range[1]
+    return {"workload": "%s: B=%d hidden=%d Hq=%d Hkv=%d D=%d theta=%g, cached tokens %s, "
+                        "%d-token blocks, tiers %s" % (cfg.name, cfg.B, cfg.H, cfg.Hq, cfg.Hkv, cfg.D,
+                                                       cfg.theta, cfg.ctx or cfg.ctx_range, cfg.T,
+                                                       cfg.tier_policy),
+            "global_batch": cfg.B * world, "seq_len": seq_len, "parallelism": "replicas x%d" % world}
+
+
 def run_reference(args, rank, world):
     cfg = WL.CONFIGS[args.config]
     if rank != 0:
@@ -342,8 +352,7 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": cfg.name, "B": cfg.B, "hidden": cfg.H, "Hq": cfg.Hq, "Hkv": cfg.Hkv,
-                       "head_dim": cfg.D, "step_sample": "1 sequence of the workload per step"},
+            "config": dict(workload_config(cfg, 1), step_sample="1 sequence of the workload per step"),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
                              "sample": "1 of %d sequences per step (full context)" % cfg.B},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -834,13 +843,8 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "%s: B=%d hidden=%d Hq=%d Hkv=%d D=%d theta=%g, cached tokens %s, "
-                               "%d-token blocks, tiers %s" % (cfg.name, cfg.B, cfg.H, cfg.Hq, cfg.Hkv, cfg.D,
-                                                              cfg.theta, cfg.ctx or cfg.ctx_range, cfg.T,
-                                                              cfg.tier_policy),
-                   "global_batch": cfg.B * world, "seq_len": cfg.ctx or max(wl.lay.seq_lens),
-                   "parallelism": "replicas x%d" % world, "attn_splits": wl.splits,
-                   "l2": "inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)},
+        "config": dict(workload_config(cfg, world), attn_splits=wl.splits,
+                       l2="inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)),
         "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
         "stage_ms": {"project": stage_ms[0], "attend_and_combine": stage_ms[1],
                      "timing": "each kernel alone (serial launches); the step overlaps them"},
