@@ -326,6 +326,20 @@ def cpu_baseline(cfg, seed, budget_s):
 # --------------------------------------------------------------------------- main
 
 
+def step_roofline(wl, ms: float, hbm_peak: float, peak_kind: str) -> dict:
+    """The decode step as a whole: algorithmic bytes per step over the step time, against
+    the HBM peak (all-HBM workloads) or the host link (host-tier bytes dominate)."""
+    c = wl.cfg
+    small = c.B * c.H * 2 + wl.new_kv_bytes + c.B * c.Hq * c.D * 2  # x, new K/V rows, out
+    hbm_bytes = wl.kv_hbm_bytes + wl.w_bytes + small
+    if wl.kv_host_bytes:
+        return {"bound": "host_link", "host_bytes": wl.kv_host_bytes, "hbm_bytes": hbm_bytes,
+                "achieved_host_gbs": wl.kv_host_bytes / (ms * 1e-3) / 1e9}
+    achieved = hbm_bytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "bytes": hbm_bytes, "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+            "frac": achieved / hbm_peak, "peak_source": peak_kind}
+
+
 def workload_config(cfg: WL.DecodeConfig, world: int) -> dict:
     """The `config` object both arms report for a decode workload."""
     seq_len = cfg.ctx or cfg.ctx_range[1]
@@ -846,6 +860,9 @@ def main():
         "config": dict(workload_config(cfg, world), attn_splits=wl.splits,
                        l2="inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)),
         "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
+        # the whole step against the same peak: every byte it must move (cached KV, W, x,
+        # the new K/V rows, out) over the step time (host-tier bytes over the host link)
+        "step_roofline": step_roofline(wl, ms, peak, peak_kind),
         "stage_ms": {"project": stage_ms[0], "attend_and_combine": stage_ms[1],
                      "timing": "each kernel alone (serial launches); the step overlaps them"},
         "roofline": ({"bound": "hbm", "kernel": "attn_mma_kernel",
