@@ -45,6 +45,8 @@ def parse():
                     help="host-tier configs: also time swap-in (DMA and copy kernel) + HBM attention")
     ap.add_argument("--attn-splits", type=int, default=0)
     ap.add_argument("--proj-splits", type=int, default=0)
+    ap.add_argument("--attn-variant", type=int, default=0,
+                    help="attention kernel (dkv_tuning.attn_variant; 6/7 = the opt-in tensor-core consumer)")
     ap.add_argument("--host-flags", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
@@ -724,7 +726,7 @@ def main():
         import dataclasses
         cfg = dataclasses.replace(cfg, B=args.batch)
     wl = Workload(cfg, seed=rank, host_flags=args.host_flags)
-    wl.set_tuning(args.attn_splits, args.proj_splits)
+    wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant)
 
     def barrier():
         if dist:
@@ -772,7 +774,7 @@ def main():
 
     # ---- per-stage durations: the same steps launched serially (no programmatic dependent
     # launch, so each kernel runs alone), with events between the two launches
-    wl.set_tuning(args.attn_splits, args.proj_splits, serial_launch=1)
+    wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant, serial_launch=1)
     for _ in range(3):
         wl.step()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
@@ -782,7 +784,7 @@ def main():
     barrier()
     stage_ms = [sum(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)) / args.steps
                 for k in range(2)]
-    wl.set_tuning(args.attn_splits, args.proj_splits)
+    wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant)
 
     # ---- e2e: host buffers in, result out, through the public API. As a serving loop runs
     # it: step k+1's inputs are copied from pinned host memory on a copy stream into the
@@ -857,7 +859,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(cfg, world), attn_splits=wl.splits,
+        "config": dict(workload_config(cfg, world), attn_splits=wl.splits, attn_variant=args.attn_variant,
                        l2="inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)),
         "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
         # the whole step against the same peak: every byte it must move (cached KV, W, x,
@@ -865,13 +867,13 @@ def main():
         "step_roofline": step_roofline(wl, ms, peak, peak_kind),
         "stage_ms": {"project": stage_ms[0], "attend_and_combine": stage_ms[1],
                      "timing": "each kernel alone (serial launches); the step overlaps them"},
-        "roofline": ({"bound": "hbm", "kernel": "attn_mma_kernel",
+        "roofline": ({"bound": "hbm", "kernel": "attn_splitk_kernel",
                       "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                       "peak_source": peak_kind,
                       "traffic": profiled_traffic(cfg.name),
                       "algorithmic_bytes_per_launch": wl.kv_bytes}
                      if not wl.kv_host_bytes else
-                     {"bound": "host_link", "kernel": "attn_mma_kernel",
+                     {"bound": "host_link", "kernel": "attn_splitk_kernel",
                       "achieved": host_info["achieved_gbs"], "peak": host_info["h2d_peak_gbs"], "unit": "GB/s",
                       "frac": host_info["frac"], "peak_source": "measured cudaMemcpy H2D (pinned, 1 GiB) in this run",
                       "traffic": None, "algorithmic_bytes_per_launch": wl.kv_host_bytes}),

@@ -19,15 +19,19 @@
 //
 // Scores are in the log2 domain: q arrives pre-scaled by log2(e)/sqrt(D), so p = 2^(s - m).
 // Two consumer implementations:
-//  * tensor cores (default): per block, S = Q.K^T and O^T += V^T.P^T as m16n8k16 bf16
-//    mma.sync with fp32 accumulation. The G query rows of a kv head are padded to the
+//  * CUDA cores (the default = variant 1; variant 2 keeps q in shared memory): packed
+//    fp32x2 FMAs. A decode query group is G <= 8 rows, G flops per KV byte: an HBM-bound
+//    product, not a dense contraction, and the tensor cores are kept for the projection.
+//  * tensor cores (opt-in, variants 6 and 7): per block, S = Q.K^T and O^T += V^T.P^T as
+//    m16n8k16 bf16 mma.sync with fp32 accumulation. The G query rows of a kv head are padded to the
 //    16-row tile, and the spare rows carry the bf16 low parts: q = q_hi + q_lo (rows
 //    0..G-1 and 8..8+G-1) and p = p_hi + p_lo (separate columns), so the products keep
 //    about 16 significant bits of the fp32 q and p. A decode step is HBM-bound at G
-//    flops per KV byte; the tensor cores are used because they turn ~800 issued
-//    instructions per block into ~100, which is what kept the CUDA-core version from
-//    the memory roofline. Stages use the TMA 128-byte swizzle, so ldmatrix is conflict-free.
-//  * CUDA cores (variant 1, kept as the comparison point): packed fp32x2 FMAs.
+//    flops per KV byte; on the tensor cores ~800 issued instructions per block become
+//    ~100, and this consumer measured faster on B200. But padding the query rows to the
+//    tensor-core tile is exactly the reshaping of an HBM-bound product into a GEMM that
+//    this design otherwise avoids, so it stays opt-in. Its stages use the TMA 128-byte
+//    swizzle, so ldmatrix is conflict-free.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <string.h>
@@ -292,10 +296,12 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
     mbar_wait_bounded(&full[j % NST], (j / NST) & 1, pool.status, 100000000ull);
 }
 
-template <int D, int HPW, int WPB, int NST, int MINB>
+// QS: keep q in shared memory instead of registers (fewer registers, more CTAs per SM).
+template <int D, int HPW, int WPB, int NST, int MINB, bool QS>
 __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
     attn_splitk_kernel(const AttnParams p) {
   using C = AttnCfg<D, HPW, WPB, NST>;
+  constexpr int OFF_Q = (C::SMEM + 15) / 16 * 16;  // q area (QS only): [G][QCH][2][8][4] fp32
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* stages = reinterpret_cast<uint16_t*>(smem);
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
@@ -307,12 +313,14 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const PoolView& pool = p.pool;
-  // everything read below (tables, q, counters) comes from the kernels ahead in the stream
-  griddep_wait();
+  // Behind this step's projection (p.early_kv) only the consumers wait for it, before q;
+  // the producer streams the cached blocks at once (see attn_mma_kernel for why that is
+  // safe). Behind anything else every thread waits first.
+  if (!p.early_kv) griddep_wait();
   if (threadIdx.x == 0) griddep_launch_dependents();
 
   // cached tokens of this sequence, clamped to what the table can hold
-  int ctx = p.seq_lens[b];
+  int ctx = __ldcg(p.seq_lens + b);
   if (ctx < 0 || ctx / kT + 1 > p.max_blocks) {
     if (threadIdx.x == 0 && s == 0 && g == 0) flag_error(pool.status, kErrCtxTooLong);
     ctx = ctx < 0 ? 0 : min(ctx, p.max_blocks * kT);
@@ -340,22 +348,35 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
   // -------------------------------------------------------------------- consumers
   const int slot = warp / WPB, hq = warp % WPB;
   const int tg = lane >> 3, dg = lane & 7;
+  griddep_wait();  // q, k_hat, v_hat and the counters are the projection's
   const int hbase = g * C::G + hq * HPW;  // first global q head of this warp
 
-  // q of this lane's key dims, as (even, odd) dim pairs for the packed fp32x2 FMA
-  float2 q2[HPW][C::QCH][4];
-#pragma unroll
-  for (int h = 0; h < HPW; ++h)
-#pragma unroll
-    for (int hh = 0; hh < C::QCH; ++hh) {
-      const float4* src = reinterpret_cast<const float4*>(
-          p.qs + ((int64_t)b * p.Hq + hbase + h) * D + (dg + 8 * hh) * 8);
-      const float4 a = src[0], c = src[1];
-      q2[h][hh][0] = make_float2(a.x, a.y);
-      q2[h][hh][1] = make_float2(a.z, a.w);
-      q2[h][hh][2] = make_float2(c.x, c.y);
-      q2[h][hh][3] = make_float2(c.z, c.w);
+  // q of this lane's key dims, as (even, odd) dim pairs for the packed fp32x2 FMA: in
+  // registers, or (QS) in shared memory laid out [head][hh][half][dg][4] so that the eight
+  // dg lanes read 128 contiguous bytes.
+  float2 q2[QS ? 1 : HPW][QS ? 1 : C::QCH][4];
+  float* qsm = reinterpret_cast<float*>(smem + OFF_Q);
+  if constexpr (QS) {
+    for (int e = threadIdx.x; e < C::G * D; e += C::NCW * 32) {
+      const int h = e / D, d = e % D, c = d / 8, w = d % 8;
+      qsm[(((h * C::QCH + c / 8) * 2 + w / 4) * 8 + c % 8) * 4 + w % 4] =
+          p.qs[((int64_t)b * p.Hq + g * C::G + h) * D + d];
     }
+    named_bar_sync(1, C::NCW * 32);
+  } else {
+#pragma unroll
+    for (int h = 0; h < HPW; ++h)
+#pragma unroll
+      for (int hh = 0; hh < C::QCH; ++hh) {
+        const float4* src = reinterpret_cast<const float4*>(
+            p.qs + ((int64_t)b * p.Hq + hbase + h) * D + (dg + 8 * hh) * 8);
+        const float4 a = src[0], c = src[1];
+        q2[h][hh][0] = make_float2(a.x, a.y);
+        q2[h][hh][1] = make_float2(a.z, a.w);
+        q2[h][hh][2] = make_float2(c.x, c.y);
+        q2[h][hh][3] = make_float2(c.z, c.w);
+      }
+  }
 
   constexpr int NP = C::DPL / 2;  // value-dim pairs per lane
   float2 acc2[HPW][NP];
@@ -382,24 +403,55 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
       float2 v2[C::NV];
 #pragma unroll
       for (int x = 0; x < C::NV; ++x) v2[x] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int i4 = 0; i4 < 4; ++i4) {
-        const int t = tg + 4 * i4;
+      if constexpr (QS) {
 #pragma unroll
         for (int hh = 0; hh < C::QCH; ++hh) {
-          const uint4 w = *reinterpret_cast<const uint4*>(Ks + t * D + (dg + 8 * hh) * 8);
-          const float2 k0 = make_float2(bf16lo(w.x), bf16hi(w.x));
-          const float2 k1 = make_float2(bf16lo(w.y), bf16hi(w.y));
-          const float2 k2 = make_float2(bf16lo(w.z), bf16hi(w.z));
-          const float2 k3 = make_float2(bf16lo(w.w), bf16hi(w.w));
+          float2 kk[4][4];
+#pragma unroll
+          for (int i4 = 0; i4 < 4; ++i4) {
+            const uint4 w = *reinterpret_cast<const uint4*>(Ks + (tg + 4 * i4) * D + (dg + 8 * hh) * 8);
+            kk[i4][0] = make_float2(bf16lo(w.x), bf16hi(w.x));
+            kk[i4][1] = make_float2(bf16lo(w.y), bf16hi(w.y));
+            kk[i4][2] = make_float2(bf16lo(w.z), bf16hi(w.z));
+            kk[i4][3] = make_float2(bf16lo(w.w), bf16hi(w.w));
+          }
 #pragma unroll
           for (int h = 0; h < HPW; ++h) {
-            float2 a = v2[h * 4 + i4];
-            a = __ffma2_rn(q2[h][hh][0], k0, a);
-            a = __ffma2_rn(q2[h][hh][1], k1, a);
-            a = __ffma2_rn(q2[h][hh][2], k2, a);
-            a = __ffma2_rn(q2[h][hh][3], k3, a);
-            v2[h * 4 + i4] = a;
+            const float4* qp = reinterpret_cast<const float4*>(qsm) + (((hq * HPW + h) * C::QCH + hh) * 2) * 8 + dg;
+            const float4 qa = qp[0], qb = qp[8];
+            const float2 q0 = make_float2(qa.x, qa.y), q1 = make_float2(qa.z, qa.w);
+            const float2 q2b = make_float2(qb.x, qb.y), q3 = make_float2(qb.z, qb.w);
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) {
+              float2 a = v2[h * 4 + i4];
+              a = __ffma2_rn(q0, kk[i4][0], a);
+              a = __ffma2_rn(q1, kk[i4][1], a);
+              a = __ffma2_rn(q2b, kk[i4][2], a);
+              a = __ffma2_rn(q3, kk[i4][3], a);
+              v2[h * 4 + i4] = a;
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          const int t = tg + 4 * i4;
+#pragma unroll
+          for (int hh = 0; hh < C::QCH; ++hh) {
+            const uint4 w = *reinterpret_cast<const uint4*>(Ks + t * D + (dg + 8 * hh) * 8);
+            const float2 k0 = make_float2(bf16lo(w.x), bf16hi(w.x));
+            const float2 k1 = make_float2(bf16lo(w.y), bf16hi(w.y));
+            const float2 k2 = make_float2(bf16lo(w.z), bf16hi(w.z));
+            const float2 k3 = make_float2(bf16lo(w.w), bf16hi(w.w));
+#pragma unroll
+            for (int h = 0; h < HPW; ++h) {
+              float2 a = v2[h * 4 + i4];
+              a = __ffma2_rn(q2[h][hh][0], k0, a);
+              a = __ffma2_rn(q2[h][hh][1], k1, a);
+              a = __ffma2_rn(q2[h][hh][2], k2, a);
+              a = __ffma2_rn(q2[h][hh][3], k3, a);
+              v2[h * 4 + i4] = a;
+            }
           }
         }
       }
@@ -818,11 +870,11 @@ static int launch_pdl(void (*fn)(KArgs...), dim3 grid, int threads, int smem, cu
   return cuda_check(cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...), "attention launch");
 }
 
-template <int D, int HPW, int WPB, int NST, int MINB>
+template <int D, int HPW, int WPB, int NST, int MINB, bool QS = false>
 static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
   using C = AttnCfg<D, HPW, WPB, NST>;
-  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB>;
-  constexpr int smem = C::SMEM;
+  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB, QS>;
+  constexpr int smem = QS ? (C::SMEM + 15) / 16 * 16 + C::G * D * 4 : C::SMEM;
   static bool attr_done = false;  // per instantiation
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -856,12 +908,13 @@ static int launch_attn_mma(const AttnParams& p, int B, int Hkv, cudaStream_t st)
 }
 
 // Kernel per (D, G) and variant:
-//   0 automatic = 6: tensor cores, 4-stage ring (one stage per consumer slot), four CTAs
-//     per SM (G = 8: 12 stages, two CTAs per SM); measured best on B200 for the 8B-shaped
-//     HBM layer (more resident CTAs beat deeper rings: 6.55 vs 6.16 TB/s)
-//   7: tensor cores, 8-stage ring, three CTAs per SM (G <= 4)
+//   0 automatic = 1 (the tensor cores are reserved for the projection)
 //   1: CUDA cores, q in registers, 8-stage ring, three CTAs per SM (G = 8: two warps per
 //      block, one CTA per SM)
+//   2: CUDA cores, q in shared memory, 4-stage ring (one stage per consumer slot), four
+//      CTAs per SM (G <= 4)
+//   6: tensor cores, 4-stage ring, four CTAs per SM (G = 8: 12 stages, two CTAs per SM)
+//   7: tensor cores, 8-stage ring, three CTAs per SM (G <= 4)
 // (Rings must be a multiple of the four consumer slots.)
 template <int D>
 static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant, cudaStream_t st) {
@@ -872,7 +925,7 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
       case 4: return launch_attn_mma<D, 4, 8, 3>(p, B, Hkv, st);
     }
   }
-  if (variant == 0 || variant == 6 || variant == 7) {
+  if (variant == 6 || variant == 7) {
     switch (G) {
       case 1: return launch_attn_mma<D, 1, 4, 4>(p, B, Hkv, st);
       case 2: return launch_attn_mma<D, 2, 4, 4>(p, B, Hkv, st);
@@ -880,6 +933,14 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
       case 8: return launch_attn_mma<D, 8, 12, 2>(p, B, Hkv, st);
     }
     return set_error(DKV_ERR_UNSUPPORTED, "attention: unsupported G=%d", G);
+  }
+  if (variant == 2) {
+    switch (G) {
+      case 1: return launch_attn_t<D, 1, 1, 4, 4, true>(p, B, Hkv, st);
+      case 2: return launch_attn_t<D, 2, 1, 4, 4, true>(p, B, Hkv, st);
+      case 4: return launch_attn_t<D, 4, 1, 4, 4, true>(p, B, Hkv, st);
+      default: break;  // G = 8: the variant-1 shape
+    }
   }
   switch (G) {
     case 1: return launch_attn_t<D, 1, 1, 8, 3>(p, B, Hkv, st);
@@ -891,8 +952,9 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
 }
 
 int attention_ctas_per_sm(int G, int variant) {
-  if (variant == 0 || variant == 6) return G == 8 ? 2 : 4;
+  if (variant == 6) return G == 8 ? 2 : 4;
   if (variant == 7) return G == 8 ? 2 : 3;
+  if (variant == 2) return G == 8 ? 1 : 4;
   return G == 8 ? 1 : 3;
 }
 

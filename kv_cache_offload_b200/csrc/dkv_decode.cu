@@ -27,7 +27,7 @@ static int pick_attn_splits(const dkv_pool* pool, int B, int Hkv, int G, int max
     const int variant = pool->tuning.attn_variant;
     const int slots = pool->num_sms * attention_ctas_per_sm(G, variant);
     const int units = B * Hkv;
-    if (variant == 0 || variant == 6 || variant == 7) {
+    if (variant == 6 || variant == 7) {
       s = (7 * slots + 4 * units) / (8 * units);  // round(7/8 * slots / units)
       if (s > 32) s = 32;
     } else {
