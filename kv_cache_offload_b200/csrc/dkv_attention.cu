@@ -495,6 +495,7 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
       if (head_leader) al[h_lane] = alpha;
       __syncwarp();
       // ---- P.V: lane owns value dims [lane*DPL, lane*DPL + DPL) as packed pairs
+if (__any_sync(0xffffffffu, alpha != 1.f))  // lazy rescale: multiplying by 1 is exact
 #pragma unroll
       for (int h = 0; h < HPW; ++h) {
         const float a = al[h];
