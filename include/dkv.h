@@ -80,9 +80,11 @@ typedef struct dkv_pool_config {
 typedef struct dkv_tuning {
   int32_t attn_splits;   /* split-K factor of the attention grid (per sequence, kv head) */
   int32_t proj_splits;   /* cluster size of the projection (its reduction split), <= 16 */
-  int32_t attn_variant;  /* attention kernel: 0 automatic (= 1), 1 CUDA-core products
-                            (q in registers, 8-stage ring, 3 CTAs/SM), 2 CUDA cores with q
-                            in shared memory (4-stage ring, 4 CTAs/SM), 6 tensor-core
+  int32_t attn_variant;  /* attention kernel: 0 automatic (= 5), 5 CUDA-core products
+                            (q in registers, 3 consumer warps, 6-stage ring, 4 CTAs/SM;
+                            G = 8 runs the variant-1 shape), 1 CUDA cores with 4 consumer
+                            warps, an 8-stage ring and 3 CTAs/SM, 2 CUDA cores with q in
+                            shared memory (4-stage ring, 4 CTAs/SM), 6 tensor-core
                             products (4-stage ring, 4 CTAs/SM), 7 tensor cores with an
                             8-stage ring (3 CTAs/SM); other values are invalid. The
                             tensor-core consumers are opt-in: the design reserves the

@@ -12,15 +12,17 @@
 //      - host-tier block: all 32 lanes issue 16-byte cp.async loads straight from the
 //        mapped pinned host memory (coalesced 512-byte warp requests), no staging buffer;
 //    both complete on the stage's mbarrier, so the consumers see one kind of stage;
-//  * four consumer "slots" take blocks round robin, each keeping its own online-softmax
-//    state (running max m, running sum l, accumulator) in registers; the slots merge at
-//    the end and the CTA writes one partial state (m, l, acc[D]) per q head to the
-//    workspace; the last split CTA of a (sequence, kv head) merges the splits.
+//  * SL consumer "slots" (warps; three in the default shape, four otherwise) take blocks
+//    round robin, each keeping its own online-softmax state (running max m, running sum
+//    l, accumulator) in registers; the slots merge at the end and the CTA writes one
+//    partial state (m, l, acc[D]) per q head to the workspace; the last split CTA of a
+//    (sequence, kv head) merges the splits.
 //
 // Scores are in the log2 domain: q arrives pre-scaled by log2(e)/sqrt(D), so p = 2^(s - m).
 // Two consumer implementations:
-//  * CUDA cores (the default = variant 1; variant 2 keeps q in shared memory): packed
-//    fp32x2 FMAs. A decode query group is G <= 8 rows, G flops per KV byte: an HBM-bound
+//  * CUDA cores (the default = variant 5: three slots, a 6-stage ring, four CTAs per SM;
+//    variant 1: four slots, an 8-stage ring, three CTAs per SM; variant 2 keeps q in
+//    shared memory): packed fp32x2 FMAs. A decode query group is G <= 8 rows, G flops per KV byte: an HBM-bound
 //    product, not a dense contraction, and the tensor cores are kept for the projection.
 //  * tensor cores (opt-in, variants 6 and 7): per block, S = Q.K^T and O^T += V^T.P^T as
 //    m16n8k16 bf16 mma.sync with fp32 accumulation. The G query rows of a kv head are padded to the
@@ -46,10 +48,10 @@ namespace dkv {
 constexpr int kSlots = 4;
 constexpr int kT = 16;
 
-template <int D, int HPW, int WPB, int NST>
+template <int D, int HPW, int WPB, int NST, int SL = kSlots>
 struct AttnCfg {
   static constexpr int G = HPW * WPB;
-  static constexpr int NCW = kSlots * WPB;  // consumer warps
+  static constexpr int NCW = SL * WPB;  // consumer warps
   static constexpr int THREADS = (NCW + 1) * 32;
   static constexpr int STAGE_ELEMS = 2 * kT * D;
   static constexpr int STAGE_BYTES = STAGE_ELEMS * 2;
@@ -66,10 +68,10 @@ struct AttnCfg {
   static constexpr int SMEM = OFF_BARS + 2 * NST * 8;
   static constexpr int MERGE_BYTES = NCW * HPW * D * 4 + NCW * HPW * 8;
   static_assert(MERGE_BYTES <= NST * STAGE_BYTES, "merge area must fit in the stage ring");
-  // Block i uses stage i % NST and consumer slot i % kSlots. Stage loads complete out of
+  // Block i uses stage i % NST and consumer slot i % SL. Stage loads complete out of
   // order, and a parity wait is only sound if the stage's barrier is at most one phase
   // behind the waiter; that holds when every stage belongs to a single slot.
-  static_assert(NST % kSlots == 0, "each stage must belong to exactly one consumer slot");
+  static_assert(NST % SL == 0, "each stage must belong to exactly one consumer slot");
 };
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -132,11 +134,11 @@ __device__ __forceinline__ void rs_level(float* v, bool up, int mask) {
 // base, then (m, l) per (warp, head). Merge the kSlots slots per q head, write this
 // split's partial state, and, when the launch fuses the combine, let the last split CTA of
 // (b, g) merge all S partial states in split order with the new token's term.
-template <int D, int HPW, int WPB>
+template <int D, int HPW, int WPB, int SL = kSlots>
 __device__ __forceinline__ void attn_merge_combine(const AttnParams& p, uint8_t* smem, int b, int g, int s,
                                                    int warp, int lane) {
   constexpr int G = HPW * WPB;
-  constexpr int NCW = kSlots * WPB;
+  constexpr int NCW = SL * WPB;
   const PoolView& pool = p.pool;
   const float* macc = reinterpret_cast<const float*>(smem);
   const float2* mml = reinterpret_cast<const float2*>(smem + NCW * HPW * D * 4);
@@ -145,11 +147,11 @@ __device__ __forceinline__ void attn_merge_combine(const AttnParams& p, uint8_t*
     const int wq = hh / HPW, h = hh % HPW;
     float M = -INFINITY;
 #pragma unroll
-    for (int sl = 0; sl < kSlots; ++sl) M = fmaxf(M, mml[(sl * WPB + wq) * HPW + h].x);
+    for (int sl = 0; sl < SL; ++sl) M = fmaxf(M, mml[(sl * WPB + wq) * HPW + h].x);
     float A = 0.f, Ls = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
-      for (int sl = 0; sl < kSlots; ++sl) {
+      for (int sl = 0; sl < SL; ++sl) {
         const float2 ml = mml[(sl * WPB + wq) * HPW + h];
         const float w = fast_exp2(ml.x - M);
         A = fmaf(macc[((sl * WPB + wq) * HPW + h) * D + d], w, A);
@@ -297,10 +299,10 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
 }
 
 // QS: keep q in shared memory instead of registers (fewer registers, more CTAs per SM).
-template <int D, int HPW, int WPB, int NST, int MINB, bool QS>
-__global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
+template <int D, int HPW, int WPB, int NST, int MINB, bool QS, int SL>
+__global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
     attn_splitk_kernel(const AttnParams p) {
-  using C = AttnCfg<D, HPW, WPB, NST>;
+  using C = AttnCfg<D, HPW, WPB, NST, SL>;
   constexpr int OFF_Q = (C::SMEM + 15) / 16 * 16;  // q area (QS only): [G][QCH][2][8][4] fp32
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* stages = reinterpret_cast<uint16_t*>(smem);
@@ -390,7 +392,7 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST>::THREADS, MINB)
   float2* pb = pbuf + warp * kT * HPW;   // (p, p) per (token, head)
   float* al = alph + warp * HPW;
 
-  for (int i = slot; i < n_local; i += kSlots) {
+  for (int i = slot; i < n_local; i += SL) {
     const int st = i % NST;
     if (!mbar_wait_bounded(&full[st], (i / NST) & 1, pool.status)) break;
     const int ntok = flags[st];
@@ -561,7 +563,7 @@ if (__any_sync(0xffffffffu, alpha != 1.f))  // lazy rescale: multiplying by 1 is
   if (head_leader) mml[warp * HPW + h_lane] = make_float2(m_run, l_tot);
   named_bar_sync(1, C::NCW * 32);
 
-  attn_merge_combine<D, HPW, WPB>(p, smem, b, g, s, warp, lane);
+  attn_merge_combine<D, HPW, WPB, SL>(p, smem, b, g, s, warp, lane);
 }
 
 // ------------------------------------------------------------ tensor-core consumer
@@ -871,10 +873,10 @@ static int launch_pdl(void (*fn)(KArgs...), dim3 grid, int threads, int smem, cu
   return cuda_check(cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...), "attention launch");
 }
 
-template <int D, int HPW, int WPB, int NST, int MINB, bool QS = false>
+template <int D, int HPW, int WPB, int NST, int MINB, bool QS = false, int SL = kSlots>
 static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
-  using C = AttnCfg<D, HPW, WPB, NST>;
-  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB, QS>;
+  using C = AttnCfg<D, HPW, WPB, NST, SL>;
+  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB, QS, SL>;
   constexpr int smem = QS ? (C::SMEM + 15) / 16 * 16 + C::G * D * 4 : C::SMEM;
   static bool attr_done = false;  // per instantiation
   if (!attr_done) {
@@ -909,14 +911,17 @@ static int launch_attn_mma(const AttnParams& p, int B, int Hkv, cudaStream_t st)
 }
 
 // Kernel per (D, G) and variant:
-//   0 automatic = 1 (the tensor cores are reserved for the projection)
-//   1: CUDA cores, q in registers, 8-stage ring, three CTAs per SM (G = 8: two warps per
-//      block, one CTA per SM)
+//   0 automatic = 5 (the tensor cores are reserved for the projection)
+//   5: CUDA cores, q in registers, three consumer slots with two stages each (6-stage
+//      ring), four CTAs per SM: 16 warps of 128 registers fill the register file, and
+//      four producers per SM stream HBM faster than three (G = 8: the variant-1 shape)
+//   1: CUDA cores, q in registers, four slots, 8-stage ring, three CTAs per SM (G = 8: two
+//      warps per block, one CTA per SM)
 //   2: CUDA cores, q in shared memory, 4-stage ring (one stage per consumer slot), four
 //      CTAs per SM (G <= 4)
 //   6: tensor cores, 4-stage ring, four CTAs per SM (G = 8: 12 stages, two CTAs per SM)
 //   7: tensor cores, 8-stage ring, three CTAs per SM (G <= 4)
-// (Rings must be a multiple of the four consumer slots.)
+// (Rings must be a multiple of the consumer slots.)
 template <int D>
 static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant, cudaStream_t st) {
   if (variant == 7 && G <= 4) {
@@ -934,6 +939,14 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
       case 8: return launch_attn_mma<D, 8, 12, 2>(p, B, Hkv, st);
     }
     return set_error(DKV_ERR_UNSUPPORTED, "attention: unsupported G=%d", G);
+  }
+  if (variant == 5 || variant == 0) {
+    switch (G) {
+      case 1: return launch_attn_t<D, 1, 1, 6, 4, false, 3>(p, B, Hkv, st);
+      case 2: return launch_attn_t<D, 2, 1, 6, 4, false, 3>(p, B, Hkv, st);
+      case 4: return launch_attn_t<D, 4, 1, 6, 4, false, 3>(p, B, Hkv, st);
+      default: break;  // G = 8: the variant-1 shape
+    }
   }
   if (variant == 2) {
     switch (G) {
@@ -955,7 +968,7 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
 int attention_ctas_per_sm(int G, int variant) {
   if (variant == 6) return G == 8 ? 2 : 4;
   if (variant == 7) return G == 8 ? 2 : 3;
-  if (variant == 2) return G == 8 ? 1 : 4;
+  if (variant == 2 || variant == 5 || variant == 0) return G == 8 ? 1 : 4;
   return G == 8 ? 1 : 3;
 }
 

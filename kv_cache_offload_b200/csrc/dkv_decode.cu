@@ -21,19 +21,33 @@ namespace dkv {
 // shape, B=16 x 32 K: 311 us at 4 splits vs 326 us at 13 = 2.8 waves); more waves only
 // add per-CTA setup and merge work. CUDA-core kernels: about 2.9 waves (their best).
 // Host-bound configurations are insensitive to the split count.
+static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant) {
+  const int slots = pool->num_sms * attention_ctas_per_sm(G, variant);
+  const int units = B * Hkv;
+  if (variant == 6 || variant == 7) {
+    const int s = (7 * slots + 4 * units) / (8 * units);  // round(7/8 * slots / units)
+    return s > 32 ? 32 : s;
+  }
+  return (29 * slots + 5 * units) / (10 * units);
+}
+
+// The automatic attention kernel (CUDA cores). Four CTAs per SM with three consumer slots
+// (variant 5) beat three CTAs with four slots (variant 1) on long contexts (8B shape,
+// B=16 x 32 K: step 398 vs 411 us, attention alone 354 vs 372 us), but at 2.9 waves of
+// its more numerous CTA slots it cuts short contexts into too many splits (B=4 x 32 K:
+// 54 splits of 38 blocks, 192 vs 147 us per step). So it is used when its splits keep at
+// least 100 blocks of the table each; otherwise, and for G = 8, variant 1.
+static int resolve_attn_variant(const dkv_pool* pool, int B, int Hkv, int G, int max_blocks) {
+  const int v = pool->tuning.attn_variant;
+  if (v != 0) return v;
+  if (G == 8) return 1;
+  const int s5 = pool->tuning.attn_splits > 0 ? pool->tuning.attn_splits : auto_splits(pool, B, Hkv, G, 5);
+  return max_blocks >= 100 * (s5 < 1 ? 1 : s5) ? 5 : 1;
+}
+
 static int pick_attn_splits(const dkv_pool* pool, int B, int Hkv, int G, int max_blocks) {
   int s = pool->tuning.attn_splits;
-  if (s <= 0) {
-    const int variant = pool->tuning.attn_variant;
-    const int slots = pool->num_sms * attention_ctas_per_sm(G, variant);
-    const int units = B * Hkv;
-    if (variant == 6 || variant == 7) {
-      s = (7 * slots + 4 * units) / (8 * units);  // round(7/8 * slots / units)
-      if (s > 32) s = 32;
-    } else {
-      s = (29 * slots + 5 * units) / (10 * units);
-    }
-  }
+  if (s <= 0) s = auto_splits(pool, B, Hkv, G, resolve_attn_variant(pool, B, Hkv, G, max_blocks));
   if (s > max_blocks) s = max_blocks;
   return s < 1 ? 1 : s;
 }
@@ -158,7 +172,8 @@ static int decode_attend(dkv_pool* pool, int layer, const int32_t* block_table, 
   a.lsu_hbm = pool->tuning.attn_lsu_hbm;
   a.pdl = !pool->tuning.serial_launch;
   a.early_kv = early_kv && a.pdl;
-  return launch_attention(a, B, w.Hkv, w.D, w.G, pool->tuning.attn_variant, (cudaStream_t)stream);
+  return launch_attention(a, B, w.Hkv, w.D, w.G, resolve_attn_variant(pool, B, w.Hkv, w.G, max_blocks),
+                          (cudaStream_t)stream);
 }
 }  // namespace dkv
 

@@ -202,7 +202,7 @@ def test_staged_calls_match_fused_step():
         ctx.close()
 
 
-@pytest.mark.parametrize("variant", [1, 2, 6, 7])  # 0 (automatic) is 1
+@pytest.mark.parametrize("variant", [1, 2, 5, 6, 7])  # 0 (automatic) is 1
 @pytest.mark.parametrize("splits", [1, 0])  # one split: long CTAs that wrap the stage ring
 @pytest.mark.parametrize("D", [64, 128])
 def test_attention_kernel_variants(variant, splits, D):
