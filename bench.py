@@ -860,6 +860,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(cfg, world), attn_splits=wl.splits, attn_variant=args.attn_variant,
+                       attn_kernel_variant=dkv.dkv_decode_attn_variant(wl.pool, cfg.B, wl.lay.max_blocks, cfg.Hq),
                        l2="inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)),
         "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
         # the whole step against the same peak: every byte it must move (cached KV, W, x,

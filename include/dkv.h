@@ -242,6 +242,12 @@ size_t dkv_decode_static_workspace_capacity(void);
 /* The attention split-K factor dkv_decode_step uses for this shape (after tuning). */
 int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 
+/* The attention kernel variant dkv_decode_step runs for this shape: the pool's
+ * dkv_tuning.attn_variant, or, when that is 0, the automatic choice (5 when its split-K
+ * ranges keep at least 100 blocks of the table each, else 1; 1 for Hq/Hkv = 8).
+ * Returns the variant (> 0) or a negative DKV_ERR_* code. */
+int dkv_decode_attn_variant(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
+
 /*
  * Block-layout permutation (Strata's layout decoupling with GPU-driven copy: "「KV Cache
  * 内存层级」系列总纲", §2.4 Strata): copy `src` laid out as [A][Bn][chunk] into `dst` as

@@ -93,6 +93,7 @@ _SIGS = {
     "dkv_decode_attend": (_I, [_P, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dkv_decode_combine": (_I, [_P, _I, _I, _I, _I, _P, _P, _SZ, _P]),
     "dkv_decode_attn_splits": (_I, [_P, _I, _I, _I]),
+    "dkv_decode_attn_variant": (_I, [_P, _I, _I, _I]),
     "dkv_decode_step_static": (_I, [_P, _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _P, _P]),
     "dkv_decode_static_workspace_capacity": (_SZ, []),
     "dkv_permute_layout": (_I, [_P, _P, _I, _I, _I64, _I64, _P]),
@@ -255,6 +256,13 @@ def dkv_decode_workspace_bytes(pool: int, B: int, max_blocks: int, num_q_heads: 
 
 def dkv_decode_attn_splits(pool: int, B: int, max_blocks: int, num_q_heads: int) -> int:
     r = lib().dkv_decode_attn_splits(pool, B, max_blocks, num_q_heads)
+    if r < 0:
+        raise DkvError(r, dkv_last_error())
+    return r
+
+
+def dkv_decode_attn_variant(pool: int, B: int, max_blocks: int, num_q_heads: int) -> int:
+    r = lib().dkv_decode_attn_variant(pool, B, max_blocks, num_q_heads)
     if r < 0:
         raise DkvError(r, dkv_last_error())
     return r

@@ -106,6 +106,13 @@ int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_
   return rc ? rc : w.S;
 }
 
+int dkv_decode_attn_variant(const dkv_pool* pool, int B, int max_blocks, int num_q_heads) {
+  if (!pool) return set_error(DKV_ERR_ARG, "null pool");
+  DecodeWs w;
+  int rc = decode_ws_layout(pool, B, max_blocks, num_q_heads, 64, &w);
+  return rc ? rc : resolve_attn_variant(pool, B, w.Hkv, w.G, max_blocks);
+}
+
 int dkv_decode_project(dkv_pool* pool, int layer, const uint16_t* x, const uint16_t* Wqkv,
                        const int32_t* block_table, const int32_t* seq_lens, const uint8_t* tier_map, int B,
                        int max_blocks, int hidden, int num_q_heads, float rope_theta, void* workspace,
