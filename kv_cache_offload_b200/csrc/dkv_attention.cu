@@ -80,25 +80,64 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// Merge the S split states of one (b, q head) output element with the new token's term:
+// One warp merges the n partial states of one (sequence, q head) -- entries base,
+// base + stride, ... -- with the new token's term and writes the D bf16 outputs:
 // M = max(s_new, m_s), L = 2^(s_new-M) + sum l_s 2^(m_s-M),
-// o = (v_new 2^(s_new-M) + sum acc_s 2^(m_s-M)) / L. Splits are read in index order.
-__device__ __forceinline__ float combine_value(const float2* __restrict__ ml, const float* __restrict__ acc,
-                                               int S, int64_t base, int D, int d, float sn, float vn) {
+// o_d = (v_d 2^(s_new-M) + sum acc_s[d] 2^(m_s-M)) / L.
+// Lane s (mod 32) holds the weight of entry s; L is summed over a fixed shuffle tree and
+// o over the entries in index order, so the result does not depend on which CTA merges
+// and the fused and the standalone combine produce identical bits. The accumulator loads
+// of four entries for all of a lane's D/32 dims are in flight together.
+template <int D>
+__device__ __forceinline__ void combine_head_warp(const float2* __restrict__ ml, const float* __restrict__ acc,
+                                                  int n, int64_t base, int stride, float sn,
+                                                  const float* __restrict__ vn, uint16_t* __restrict__ out,
+                                                  int lane) {
+  constexpr int DL = D / 32;
   float M = sn;
-  for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(ml + base + s).x);
-  const float wn = exp2f(sn - M);
-  float L = wn;
-  float A = wn * vn;
-  for (int s = 0; s < S; ++s) {
-    const float2 m = __ldcg(ml + base + s);
-    if (m.x != -INFINITY) {
-      const float w = exp2f(m.x - M);
-      L = fmaf(m.y, w, L);
-      A = fmaf(__ldcg(acc + (base + s) * D + d), w, A);
+  for (int s = lane; s < n; s += 32) M = fmaxf(M, __ldcg(ml + base + (int64_t)s * stride).x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float wn = exp2f(sn - M);  // M >= s_new is finite; an empty state (m = -inf) weighs 0
+  float Lp = 0.f;
+  for (int s = lane; s < n; s += 32) {
+    const float2 m = __ldcg(ml + base + (int64_t)s * stride);
+    Lp = fmaf(m.y, exp2f(m.x - M), Lp);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) Lp += __shfl_xor_sync(0xffffffffu, Lp, o);
+  const float L = wn + Lp;
+  float A[DL];
+#pragma unroll
+  for (int k = 0; k < DL; ++k) A[k] = wn * vn[lane + 32 * k];
+  for (int s0 = 0; s0 < n; s0 += 32) {
+    const int cnt = min(32, n - s0);
+    float wmine = 0.f;
+    if (lane < cnt) wmine = exp2f(__ldcg(ml + base + (int64_t)(s0 + lane) * stride).x - M);
+    int t = 0;
+    for (; t + 4 <= cnt; t += 4) {
+      float a[4][DL];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int k = 0; k < DL; ++k)
+          a[u][k] = __ldcg(acc + (base + (int64_t)(s0 + t + u) * stride) * D + lane + 32 * k);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float w = __shfl_sync(0xffffffffu, wmine, t + u);
+#pragma unroll
+        for (int k = 0; k < DL; ++k) A[k] = fmaf(a[u][k], w, A[k]);
+      }
+    }
+    for (; t < cnt; ++t) {
+      const float w = __shfl_sync(0xffffffffu, wmine, t);
+#pragma unroll
+      for (int k = 0; k < DL; ++k)
+        A[k] = fmaf(__ldcg(acc + (base + (int64_t)(s0 + t) * stride) * D + lane + 32 * k), w, A[k]);
     }
   }
-  return A / L;
+#pragma unroll
+  for (int k = 0; k < DL; ++k) out[lane + 32 * k] = f32_to_bf16_bits(A[k] / L);
 }
 
 // The new token's score s_new = q . k_hat (log2 domain: q is pre-scaled), computed by one
@@ -167,25 +206,18 @@ __device__ __forceinline__ void attn_merge_combine(const AttnParams& p, uint8_t*
   // (in split order, so the result does not depend on which CTA finishes last)
   if (p.out) {
     __shared__ int s_last;
-    __shared__ float s_new[8];
     __threadfence();
     named_bar_sync(1, NCW * 32);
     if (threadIdx.x == 0) s_last = atomicAdd(p.cnt + (int64_t)b * pool.Hkv + g, 1) == p.S - 1;
     named_bar_sync(1, NCW * 32);
-    if (s_last) {
+    if (s_last) {  // one warp per q head of the group
       __threadfence();
       const float* kn = p.knew + ((int64_t)b * pool.Hkv + g) * D;
       for (int hh = warp; hh < G; hh += NCW) {
-        const float sc = new_token_score(p.qs + ((int64_t)b * p.Hq + g * G + hh) * D, kn, D, lane);
-        if (lane == 0) s_new[hh] = sc;
-      }
-      named_bar_sync(1, NCW * 32);
-      for (int o = threadIdx.x; o < G * D; o += NCW * 32) {
-        const int hh = o / D, d = o % D;
         const int hg = g * G + hh;
-        const float r = combine_value(p.part_ml, p.part_acc, p.S, ((int64_t)b * p.Hq + hg) * p.S, D, d,
-                                      s_new[hh], p.vnew[((int64_t)b * pool.Hkv + g) * D + d]);
-        p.out[((int64_t)b * p.Hq + hg) * D + d] = f32_to_bf16_bits(r);
+        const float sn = new_token_score(p.qs + ((int64_t)b * p.Hq + hg) * D, kn, D, lane);
+        combine_head_warp<D>(p.part_ml, p.part_acc, p.S, ((int64_t)b * p.Hq + hg) * p.S, 1, sn,
+                             p.vnew + ((int64_t)b * pool.Hkv + g) * D, p.out + ((int64_t)b * p.Hq + hg) * D, lane);
       }
       if (threadIdx.x == 0) p.cnt[(int64_t)b * pool.Hkv + g] = 0;
     }
@@ -832,25 +864,18 @@ __global__ void __launch_bounds__((kSlots + 1) * 32, MINB)
 
 // out[b][h] = (sum_s acc_s 2^(m_s-M) + v_new 2^(s_new-M)) / (sum_s l_s 2^(m_s-M) + 2^(s_new-M))
 // over the S split partials and the new token's (score s_new, value v_hat); bf16 RNE.
+// The standalone combine (after attend(out = nullptr)): one warp per (q head, sequence),
+// the same merge as the fused combine.
 template <int D>
-__global__ void __launch_bounds__(D) combine_kernel(int Hq, int Hkv, int S,
-                                                    const float2* __restrict__ ml,
-                                                    const float* __restrict__ acc,
-                                                    const float* __restrict__ qs,
-                                                    const float* __restrict__ knew,
-                                                    const float* __restrict__ vnew,
-                                                    uint16_t* __restrict__ out) {
-  const int hg = blockIdx.x, b = blockIdx.y, d = threadIdx.x;
+__global__ void __launch_bounds__(32) combine_kernel(int Hq, int Hkv, int S, const float2* __restrict__ ml,
+                                                     const float* __restrict__ acc, const float* __restrict__ qs,
+                                                     const float* __restrict__ knew, const float* __restrict__ vnew,
+                                                     uint16_t* __restrict__ out) {
+  const int hg = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
   const int g = hg / (Hq / Hkv);
-  __shared__ float s_new;
-  if (d < 32) {
-    const float sc = new_token_score(qs + ((int64_t)b * Hq + hg) * D, knew + ((int64_t)b * Hkv + g) * D, D, d);
-    if (d == 0) s_new = sc;
-  }
-  __syncthreads();
-  const float r = combine_value(ml, acc, S, ((int64_t)b * Hq + hg) * S, D, d, s_new,
-                                vnew[((int64_t)b * Hkv + g) * D + d]);
-  out[((int64_t)b * Hq + hg) * D + d] = f32_to_bf16_bits(r);
+  const float sn = new_token_score(qs + ((int64_t)b * Hq + hg) * D, knew + ((int64_t)b * Hkv + g) * D, D, lane);
+  combine_head_warp<D>(ml, acc, S, ((int64_t)b * Hq + hg) * S, 1, sn, vnew + ((int64_t)b * Hkv + g) * D,
+                       out + ((int64_t)b * Hq + hg) * D, lane);
 }
 
 // ---------------------------------------------------------------------- launchers
@@ -982,9 +1007,9 @@ int launch_combine(int B, int Hq, int Hkv, int D, int S, const float2* ml, const
                    const float* qs, const float* knew, const float* vnew, uint16_t* out, cudaStream_t st) {
   dim3 grid(Hq, B);
   if (D == 128)
-    combine_kernel<128><<<grid, 128, 0, st>>>(Hq, Hkv, S, ml, acc, qs, knew, vnew, out);
+    combine_kernel<128><<<grid, 32, 0, st>>>(Hq, Hkv, S, ml, acc, qs, knew, vnew, out);
   else
-    combine_kernel<64><<<grid, 64, 0, st>>>(Hq, Hkv, S, ml, acc, qs, knew, vnew, out);
+    combine_kernel<64><<<grid, 32, 0, st>>>(Hq, Hkv, S, ml, acc, qs, knew, vnew, out);
   return cuda_check(cudaGetLastError(), "combine launch");
 }
 
