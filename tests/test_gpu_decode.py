@@ -83,6 +83,23 @@ def test_step_is_repeatable():
         ctx.close()
 
 
+def test_automatic_attention_variant():
+    """The automatic choice between the two CUDA-core shapes (148 SMs): the four-CTA shape
+    while its splits keep >= 100 table blocks each, else (and for G = 8) the three-CTA one;
+    an explicit tuning value is taken as is."""
+    pool = dkv.dkv_pool_create(1, 8, 128, 4, 1, block_tokens=16)
+    try:
+        assert dkv.dkv_decode_attn_variant(pool, 16, 2050, 32) == 5
+        assert dkv.dkv_decode_attn_splits(pool, 16, 2050, 32) == 13
+        assert dkv.dkv_decode_attn_variant(pool, 4, 2050, 32) == 1
+        assert dkv.dkv_decode_attn_splits(pool, 4, 2050, 32) == 40
+        assert dkv.dkv_decode_attn_variant(pool, 16, 2050, 64) == 1
+        dkv.dkv_pool_set_tuning(pool, attn_variant=7)
+        assert dkv.dkv_decode_attn_variant(pool, 16, 2050, 32) == 7
+    finally:
+        dkv.dkv_pool_destroy(pool)
+
+
 def test_bad_table_entries_are_flagged_not_fatal():
     cfg = WL.small_config(B=2, ctx_range=(40, 60), host_prob=0.5)
     inp = WL.make_decode_inputs(cfg)
