@@ -170,7 +170,7 @@ __device__ __forceinline__ void rs_level(float* v, bool up, int mask) {
 
 // ------------------------------------------------------------- slot merge + combine
 // The consumer slots have left their state in shared memory: acc [NCW*HPW][D] fp32 at the
-// base, then (m, l) per (warp, head). Merge the kSlots slots per q head, write this
+// base, then (m, l) per (warp, head). Merge the SL slots per q head, write this
 // split's partial state, and, when the launch fuses the combine, let the last split CTA of
 // (b, g) merge all S partial states in split order with the new token's term.
 template <int D, int HPW, int WPB, int SL = kSlots>
@@ -577,7 +577,7 @@ if (__any_sync(0xffffffffu, alpha != 1.f))  // lazy rescale: multiplying by 1 is
     if (lane == 0) mbar_arrive(&empty[st]);
   }
 
-  // ---- per-warp totals of l, then merge the four slots through shared memory
+  // ---- per-warp totals of l, then merge the SL slots through shared memory
   float l_tot = l_run;
 #pragma unroll
   for (int mask = 1; mask <= C::LOWMASK; mask <<= 1) l_tot += __shfl_xor_sync(0xffffffffu, l_tot, mask);
