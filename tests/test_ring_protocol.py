@@ -53,10 +53,13 @@ def _run(nst, slots, n, seed):
 
 
 def test_ring_used_by_the_kernel_is_sound():
-    for nst in (8, 12):
+    # (stages, slots) of the kernel shapes: four slots with 8 (three CTAs per SM) or 4/12
+    # stages (the tensor-core consumer), three slots with 6 stages (four CTAs per SM)
+    for nst, slots in ((8, 4), (12, 4), (4, 4), (6, 3)):
         for seed in range(1500):
-            assert _run(nst, 4, 48, seed) is None, (nst, seed)
+            assert _run(nst, slots, 48, seed) is None, (nst, slots, seed)
 
 
 def test_ring_that_is_not_a_multiple_of_the_slots_is_unsound():
     assert any(_run(6, 4, 48, seed) for seed in range(200))
+    assert any(_run(8, 3, 48, seed) for seed in range(200))
