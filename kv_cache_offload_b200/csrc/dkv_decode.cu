@@ -35,8 +35,9 @@ static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant)
 // (variant 5) beat three CTAs with four slots (variant 1) on long contexts (8B shape,
 // B=16 x 32 K: step 398 vs 411 us, attention alone 354 vs 372 us), but at 2.9 waves of
 // its more numerous CTA slots it cuts short contexts into too many splits (B=4 x 32 K:
-// 54 splits of 38 blocks, 192 vs 147 us per step). So it is used when its splits keep at
-// least 100 blocks of the table each; otherwise, and for G = 8, variant 1.
+// 54 splits of 38 blocks, 192 vs 147 us per step; both comparisons measured before the
+// split merge was batched). So it is used when its splits keep at least 100 blocks of the
+// table each; otherwise, and for G = 8, variant 1.
 static int resolve_attn_variant(const dkv_pool* pool, int B, int Hkv, int G, int max_blocks) {
   const int v = pool->tuning.attn_variant;
   if (v != 0) return v;
