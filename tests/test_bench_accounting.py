@@ -1,0 +1,49 @@
+"""The benchmark's byte accounting and its reported fields, on the CPU.
+
+The step roofline counts every byte a decode step must move once: the cached KV, the
+QKV weight, x, the new K/V rows and the output. For the 8B-shaped all-HBM workload
+(B=16, 32768 cached tokens, Hq/Hkv = 32/8, D=128, hidden 4096) that is
+2^31 + 50,331,648 + 131,072 + 65,536 + 131,072 = 2,198,142,976 bytes.
+"""
+from types import SimpleNamespace
+
+import pytest
+
+import bench
+import workloads as WL
+
+
+def _wl(host_bytes=0):
+    cfg = WL.CONFIGS["8b_hbm"]
+    kv = cfg.B * cfg.ctx * cfg.Hkv * 2 * cfg.D * 2
+    return SimpleNamespace(cfg=cfg, kv_hbm_bytes=kv - host_bytes, kv_host_bytes=host_bytes,
+                           w_bytes=(cfg.Hq + 2 * cfg.Hkv) * cfg.D * cfg.H * 2,
+                           new_kv_bytes=cfg.B * cfg.Hkv * cfg.D * 2 * 2)
+
+
+def test_step_roofline_bytes_for_the_8b_layer():
+    wl = _wl()
+    assert wl.kv_hbm_bytes == 2 ** 31 and wl.w_bytes == 50331648
+    r = bench.step_roofline(wl, 0.4, 6543.4, "measured")
+    assert r["bound"] == "hbm" and r["bytes"] == 2198142976
+    assert r["achieved"] == pytest.approx(2198142976 / 0.4e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6543.4)
+
+
+def test_step_roofline_is_host_bound_when_blocks_live_on_the_host():
+    wl = _wl(host_bytes=2 ** 30)
+    r = bench.step_roofline(wl, 20.0, 6543.4, "measured")
+    assert r["bound"] == "host_link" and r["host_bytes"] == 2 ** 30
+    assert r["achieved_host_gbs"] == pytest.approx(2 ** 30 / 20e-3 / 1e9)
+
+
+def test_replica_throughput_counts_all_ranks_over_the_slowest():
+    assert bench.replica_throughput(16, 1, 0.4) == pytest.approx(40000.0)
+    assert bench.replica_throughput(16, 8, 0.5) == pytest.approx(16 * 8 / 0.5e-3)
+
+
+def test_workload_config_names_the_workload_without_model_keys():
+    c = bench.workload_config(WL.CONFIGS["8b_hbm"], 2)
+    assert c["global_batch"] == 32 and c["seq_len"] == 32768 and c["parallelism"] == "replicas x2"
+    assert c["workload"].startswith("8b_hbm: B=16 hidden=4096 Hq=32 Hkv=8 D=128")
+    assert "model" not in c
