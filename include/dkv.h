@@ -80,10 +80,11 @@ typedef struct dkv_pool_config {
 typedef struct dkv_tuning {
   int32_t attn_splits;   /* split-K factor of the attention grid (per sequence, kv head) */
   int32_t proj_splits;   /* cluster size of the projection (its reduction split), <= 16 */
-  int32_t attn_variant;  /* attention kernel: 0 automatic (= 5), 5 CUDA-core products
-                            (q in registers, 3 consumer warps, 6-stage ring, 4 CTAs/SM;
-                            G = 8 runs the variant-1 shape), 1 CUDA cores with 4 consumer
-                            warps, an 8-stage ring and 3 CTAs/SM, 2 CUDA cores with q in
+  int32_t attn_variant;  /* attention kernel: 0 automatic (see dkv_decode_attn_variant),
+                            5 CUDA-core products (q in registers, 3 consumer warps,
+                            6-stage ring, 4 CTAs/SM; G = 8 runs the variant-1 shape),
+                            1 CUDA cores with 4 consumer warps, an 8-stage ring and
+                            3 CTAs/SM, 2 CUDA cores with q in
                             shared memory (4-stage ring, 4 CTAs/SM), 6 tensor-core
                             products (4-stage ring, 4 CTAs/SM), 7 tensor cores with an
                             8-stage ring (3 CTAs/SM); other values are invalid. The
@@ -243,8 +244,8 @@ size_t dkv_decode_static_workspace_capacity(void);
 int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 
 /* The attention kernel variant dkv_decode_step runs for this shape: the pool's
- * dkv_tuning.attn_variant, or, when that is 0, the automatic choice (5 when its split-K
- * ranges keep at least 100 blocks of the table each, else 1; 1 for Hq/Hkv = 8).
+ * dkv_tuning.attn_variant, or, when that is 0, the automatic choice (for Hq/Hkv = 4: 5 when
+ * its split-K ranges keep at least 100 blocks of the table each, else 1; 1 otherwise).
  * Returns the variant (> 0) or a negative DKV_ERR_* code. */
 int dkv_decode_attn_variant(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 

@@ -36,12 +36,12 @@ static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant)
 // B=16 x 32 K: step 398 vs 411 us, attention alone 354 vs 372 us), but at 2.9 waves of
 // its more numerous CTA slots it cuts short contexts into too many splits (B=4 x 32 K:
 // 54 splits of 38 blocks, 192 vs 147 us per step; both comparisons measured before the
-// split merge was batched). So it is used when its splits keep at least 100 blocks of the
-// table each; otherwise, and for G = 8, variant 1.
+// split merge was batched). So it is used for G = 4 (the measured group size) when its
+// splits keep at least 100 blocks of the table each; otherwise variant 1.
 static int resolve_attn_variant(const dkv_pool* pool, int B, int Hkv, int G, int max_blocks) {
   const int v = pool->tuning.attn_variant;
   if (v != 0) return v;
-  if (G == 8) return 1;
+  if (G != 4) return 1;
   const int s5 = pool->tuning.attn_splits > 0 ? pool->tuning.attn_splits : auto_splits(pool, B, Hkv, G, 5);
   return max_blocks >= 100 * (s5 < 1 ? 1 : s5) ? 5 : 1;
 }
