@@ -94,6 +94,12 @@ ORACLE_MUTANTS = [
     ("layout-reshape-not-transpose", "layer_first_to_page_first",
      "out[:, l] = pool[l]", "out.reshape((L, P) + pool.shape[2:])[l] = pool[l]"),
     ("gemm-wrong-index", "gemm_entries", "bf16_to_f64(Bt_bits[int(j)])", "bf16_to_f64(Bt_bits[int(i) % len(Bt_bits)])"),
+    ("gemm-bound-keeps-sign-of-a", "gemm_abs_bound", "np.abs(bf16_to_f64(A_bits[int(i)]))",
+     "bf16_to_f64(A_bits[int(i)])"),
+    ("gemm-bound-keeps-sign-of-b", "gemm_abs_bound", "np.abs(bf16_to_f64(Bt_bits[int(j)]))",
+     "bf16_to_f64(Bt_bits[int(j)])"),
+    ("gemm-bound-wrong-column", "gemm_abs_bound", "np.abs(bf16_to_f64(Bt_bits[int(j)]))",
+     "np.abs(bf16_to_f64(Bt_bits[int(i) % len(Bt_bits)]))"),
 ]
 
 

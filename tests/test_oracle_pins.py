@@ -374,3 +374,28 @@ def test_naive_zero_copy_traffic_matches_published_figure():
     for bm in (32, 128, 256):
         assert abs(O.naive_zero_copy_host_bytes(n, n, n, BM=bm) / 1e9 - g["naive_B_traffic_GB"]) > 5
     assert round(g["naive_ms"] / g["swap_ms"]) == g["slowdown"]
+
+
+def test_gemm_abs_bound_exact_on_integers():
+    # sum_k |A[i,k] B[k,j]| written out over integers (exact in fp64), mixed signs, so a
+    # bound that keeps a sign, drops a factor or reads the wrong row/column differs
+    rng = np.random.default_rng(8)
+    M, N, K = 6, 5, 41
+    A = rng.integers(-9, 10, size=(M, K))
+    B = rng.integers(-9, 10, size=(K, N))
+    a_bits = O.f64_to_bf16_rne(A.astype(np.float64))
+    bt_bits = O.f64_to_bf16_rne(B.T.astype(np.float64))
+    rows, cols = np.array([0, 5, 2, 2, 4]), np.array([4, 0, 3, 1, 4])
+    got = O.gemm_abs_bound(a_bits, bt_bits, rows, cols)
+    for n, (i, j) in enumerate(zip(rows, cols)):
+        want = sum(abs(int(A[i, k]) * int(B[k, j])) for k in range(K))
+        assert got[n] == want
+        # the triangle inequality: the bound is never below |C_ij|
+        assert got[n] >= abs(sum(int(A[i, k]) * int(B[k, j]) for k in range(K)))
+    # with every product non-negative the bound is the entry itself
+    Ap, Bp = np.abs(A), np.abs(B)
+    gp = O.gemm_abs_bound(O.f64_to_bf16_rne(Ap.astype(np.float64)), O.f64_to_bf16_rne(Bp.T.astype(np.float64)),
+                          rows, cols)
+    ep = O.gemm_entries(O.f64_to_bf16_rne(Ap.astype(np.float64)), O.f64_to_bf16_rne(Bp.T.astype(np.float64)),
+                        rows, cols)
+    assert np.array_equal(gp, ep)
