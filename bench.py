@@ -1,13 +1,18 @@
 """Benchmark: fused QKV + decode attention step on a two-tier (HBM / mapped host) paged KV cache.
 
-Default workload (N=1): the Llama-3-8B-shaped layer with the whole cache in HBM — batch 16,
-hidden 4096, 32 q / 8 kv heads, head_dim 128, RoPE theta 5e5, 32768 cached tokens per
-sequence in 16-token blocks. A step is one decode step of one layer through the C ABI
-(dkv_decode_step: projection, split-K attention, combine). Inputs are synthetic (seeded
-N(0,1) activations and KV, W ~ N(0, 1/hidden)), generated on the device.
+Default workload (N=1): the Llama-3-70B-shaped layer, the largest single-GPU configuration —
+batch 32, hidden 8192, 64 q / 8 kv heads, head_dim 128, RoPE theta 5e5, cached contexts drawn
+uniformly from 8192..65536 tokens in 16-token blocks, each block in mapped pinned host memory
+with probability 0.8 (read in place over PCIe) and in HBM otherwise. Its roofline is the host
+link. In the same run the Llama-3-8B-shaped layer with the whole cache in HBM (batch 16,
+32768 cached tokens each) is timed and reported as `hbm_line`, against the HBM roofline. A
+step is one decode step of one layer through the C ABI (dkv_decode_step: projection,
+split-K attention, combine). Inputs are synthetic (seeded N(0,1) activations and KV,
+W ~ N(0, 1/hidden)), generated on the device.
 
 Multi-GPU: every rank runs an independent replica of the workload (the step has no
-cross-GPU exchange); value = tokens of all ranks / max-over-ranks time.
+cross-GPU exchange); value = tokens of all ranks / max-over-ranks time. Each rank's host
+tier is placed on its GPU's nearest NUMA node.
 
 Prints one JSON line on rank 0. `--impl reference` times the fp64 CPU oracle instead.
 """
@@ -37,19 +42,25 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="dkv", choices=["dkv", "reference"])
-    ap.add_argument("--config", default="8b_hbm", choices=sorted(WL.CONFIGS) + ["gemm", "layout", "adaptive"])
+    ap.add_argument("--config", default="70b_mixed", choices=sorted(WL.CONFIGS) + ["gemm", "layout", "adaptive"],
+                    help="decode workload (default: the largest single-GPU configuration; the all-HBM "
+                         "8B-shaped layer is then reported beside it as hbm_line)")
+    ap.add_argument("--no-hbm-line", action="store_true", help="skip the all-HBM line of the default run")
     ap.add_argument("--compare-staged", action="store_true",
                     help="host-tier configs: also time swap-in (DMA and copy kernel) + HBM attention")
     ap.add_argument("--attn-splits", type=int, default=0)
     ap.add_argument("--proj-splits", type=int, default=0)
     ap.add_argument("--attn-variant", type=int, default=0,
                     help="attention kernel (dkv_tuning.attn_variant; 6/7 = the opt-in tensor-core consumer)")
-    ap.add_argument("--host-flags", type=int, default=0)
+    ap.add_argument("--host-flags", type=int, default=2,
+                    help="dkv_pool_config.host_flags (default DKV_HOST_NUMA_NEAREST: the host tier on the "
+                         "GPU's nearest NUMA node)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
+    ap.add_argument("--ctx", type=int, default=0, help="override the cached tokens per sequence (profiling)")
     ap.add_argument("--gemm-dim", type=int, default=0, help="override M=N=K of the GEMM study (profiling)")
     ap.add_argument("--profile", action="store_true",
                     help="warm-up + timed steps only (no clock pre-roll, e2e or CPU baseline): for ncu")
@@ -77,9 +88,10 @@ def src_hash(*names):
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(config_name: str):
-    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary, if it
-    was captured on the current kernel source (else None)."""
+def profiled_traffic(config_name: str, batch: int):
+    """Per-launch traffic of the attention kernel at a full configuration, from the committed
+    ncu summary (DRAM bytes for the all-HBM layer, PCIe read bytes for host-tier ones), if it
+    was captured on the current kernel source and describes this batch (else None)."""
     p = os.path.join(ROOT, "profiles", "attention_traffic.json")
     if not os.path.exists(p):
         return None
@@ -88,7 +100,9 @@ def profiled_traffic(config_name: str):
     e = d.get(config_name)
     if not e or e.get("src_hash") != src_hash("dkv_attention.cu", "dkv_common.cuh", "dkv_umma.cuh"):
         return None
-    return e.get("bytes_per_launch")
+    if e.get("batch") != batch:
+        return None
+    return {"bytes": e.get("bytes_per_launch"), "counter": e.get("counter")}
 
 
 class ClockSampler:
@@ -274,55 +288,149 @@ def measure_h2d_peak(dev, nbytes=1 << 30, reps=5):
 
 
 # -------------------------------------------------------------------- CPU oracle
+# The oracle is timed as it stands (one sequence per call, fp64 numpy) on the host's
+# cores: one spawned process per core, each with single-threaded BLAS and torch, each on
+# its own sequence of the workload, so the core count reported is the parallelism used.
 
 
-def oracle_sample(cfg: WL.DecodeConfig, seed: int, n_seq: int):
-    """A bounded sample of the workload for the oracle: the first n_seq sequences' shapes
-    (same lengths, tiers, block counts), generated on the host."""
-    sub = WL.DecodeConfig(cfg.name, B=n_seq, H=cfg.H, Hq=cfg.Hq, Hkv=cfg.Hkv, D=cfg.D,
+def oracle_sample(cfg: WL.DecodeConfig, seed: int, seqs):
+    """A bounded sample of the workload for the oracle: the sequences `seqs` of it (their
+    context lengths), with tiers and tables drawn by the workload's own policy, generated
+    on the host."""
+    lens_all = WL.seq_lengths(cfg, seed)
+    lens = [lens_all[b % cfg.B] for b in seqs]
+    sub = WL.DecodeConfig(cfg.name, B=len(lens), H=cfg.H, Hq=cfg.Hq, Hkv=cfg.Hkv, D=cfg.D,
                           theta=cfg.theta, ctx=cfg.ctx, ctx_range=cfg.ctx_range,
                           tier_policy=cfg.tier_policy, recent_hbm_tokens=cfg.recent_hbm_tokens,
                           host_prob=cfg.host_prob, permute=cfg.permute, layers=cfg.layers, T=cfg.T)
-    lens = WL.seq_lengths(cfg, seed)[:n_seq]
     return WL.make_decode_inputs(sub, seed=seed, seq_lens=lens)
 
 
-def time_oracle(inp, budget_s: float):
-    """Run the oracle sequence by sequence, cycling over the sample's sequences, until the
-    budget is spent (at least one sequence); tokens/s."""
-    from oracle import dkv_oracle as O
+def _oracle_args(inp):
     cfg, lay = inp.cfg, inp.layout
-    xb, Wb = WL.bf16_bits(inp.x), WL.bf16_bits(inp.W)
-    tiers = [WL.bf16_bits(inp.hbm), WL.bf16_bits(inp.host)]
-    done, t0 = 0, time.perf_counter()
-    while True:
-        O.decode_step(xb, Wb, tiers, lay.block_table.numpy(), lay.seq_lens, lay.tier_map.numpy(),
-                      cfg.Hq, cfg.Hkv, cfg.D, cfg.T, cfg.theta, batch=[done % cfg.B])
-        done += 1
-        if time.perf_counter() - t0 > budget_s:
-            break
-    el = time.perf_counter() - t0
-    return done / el, done, el
+    return (WL.bf16_bits(inp.x), WL.bf16_bits(inp.W), [WL.bf16_bits(inp.hbm), WL.bf16_bits(inp.host)],
+            lay.block_table.numpy(), lay.seq_lens, lay.tier_map.numpy(), cfg.Hq, cfg.Hkv, cfg.D, cfg.T,
+            cfg.theta)
 
 
-def oracle_threads():
+def _oracle_proc(name, seed, b, budget_s, steps, bar, q):
+    """One oracle process: single-threaded, one sequence of the workload. With `steps`, each
+    step runs between two barrier waits shared with the parent (which times the step);
+    otherwise it runs until `budget_s` of its own time is spent and reports the count."""
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        if n:
-            return int(max(n))
+        torch.set_num_threads(1)
+        from threadpoolctl import threadpool_limits
+        threadpool_limits(1)
+        from oracle import dkv_oracle as O
+        cfg = WL.CONFIGS[name]
+        a = _oracle_args(oracle_sample(cfg, seed, [b]))
+        if steps:
+            for _ in range(steps):
+                bar.wait(timeout=900)
+                O.decode_step(*a)
+                bar.wait(timeout=900)
+            q.put((b, steps, 0.0, None))
+            return
+        bar.wait(timeout=900)
+        done, t0 = 0, time.perf_counter()
+        while True:
+            O.decode_step(*a)
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        q.put((b, done, time.perf_counter() - t0, None))
+    except Exception as e:  # reported to the parent, which raises
+        try:
+            bar.abort()
+        except Exception:
+            pass
+        q.put((b, 0, 0.0, repr(e)))
+
+
+def oracle_workers(cfg: WL.DecodeConfig) -> int:
+    """Processes for the oracle: one per core this process may run on, at most 16, and no
+    more than half the available host memory allows (W in fp64 and one sequence's KV each)."""
+    n = len(os.sched_getaffinity(0))
+    per = cfg.rows * cfg.H * 10 + 3 * (cfg.ctx or cfg.ctx_range[1]) * cfg.Hkv * cfg.D * 4 + (1 << 29)
+    try:
+        import psutil
+        n = min(n, max(1, int(psutil.virtual_memory().available * 0.5 // per)))
     except Exception:
         pass
-    return 1
+    return max(1, min(n, 16))
+
+
+def run_oracle_pool(cfg: WL.DecodeConfig, seed: int, workers: int, budget_s: float = 0.0, steps: int = 0):
+    """Run the oracle in `workers` spawned processes (sequences 0..workers-1 of the workload).
+    Budget mode: returns (tokens/s summed over the processes, sequences done, seconds).
+    Steps mode: returns the wall time of each step, a step being one sequence per process."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")  # never fork a process that has a CUDA context
+    bar = ctx.Barrier(workers + 1)
+    q = ctx.Queue()
+    keep = {k: os.environ.get(k) for k in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    os.environ.update({k: "1" for k in keep})
+    try:
+        procs = [ctx.Process(target=_oracle_proc, args=(cfg.name, seed, i, budget_s, steps, bar, q), daemon=True)
+                 for i in range(workers)]
+        for p in procs:
+            p.start()
+    finally:
+        for k, v in keep.items():
+            if v is None:
+                os.environ.pop(k, None)
+            else:
+                os.environ[k] = v
+    times = []
+    try:
+        if steps:
+            for _ in range(steps):
+                bar.wait(timeout=900)
+                t0 = time.perf_counter()
+                bar.wait(timeout=900)
+                times.append(time.perf_counter() - t0)
+        else:
+            bar.wait(timeout=900)
+        res = [q.get(timeout=900) for _ in procs]
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    errs = [r[3] for r in res if r[3]]
+    if errs:
+        raise RuntimeError("oracle process failed: " + errs[0])
+    if steps:
+        return times
+    rate = sum(d / el for _, d, el, _ in res if el > 0)
+    return rate, sum(d for _, d, _, _ in res), max(el for _, _, el, _ in res)
+
+
+def oracle_single_thread_tiny(seconds: float = 1.0) -> dict:
+    """The oracle on the tiny configuration (1 sequence, 512 cached tokens) with one BLAS
+    thread, in this process."""
+    from threadpoolctl import threadpool_limits
+    from oracle import dkv_oracle as O
+    a = _oracle_args(WL.make_decode_inputs(WL.CONFIGS["tiny"], seed=0))
+    with threadpool_limits(1):
+        O.decode_step(*a)
+        done, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            O.decode_step(*a)
+            done += 1
+        el = time.perf_counter() - t0
+    return {"ms_per_step": 1e3 * el / done, "tokens_per_s": done / el, "threads": 1,
+            "workload": "tiny: B=1 hidden=256 Hq=4 Hkv=2 D=64, 512 cached tokens, all host tier"}
 
 
 def cpu_baseline(cfg, seed, budget_s):
-    n_seq = max(1, min(cfg.B, 4))
-    inp = oracle_sample(cfg, seed, n_seq)
-    rate, done, el = time_oracle(inp, budget_s)
-    return {"value": rate, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
-            "sample": "%d sequence decode steps cycling over %d of the workload's %d sequences (full "
-                      "context each), %.1f s of fp64 numpy oracle work" % (done, n_seq, cfg.B, el)}
+    workers = oracle_workers(cfg)
+    rate, done, el = run_oracle_pool(cfg, seed, workers, budget_s=budget_s)
+    return {"value": rate, "unit": "tokens/s", "cores": workers, "kind": "oracle",
+            "sample": "%d processes x 1 thread, each decoding one sequence of the workload (full context, "
+                      "sequences 0..%d) repeatedly for %.1f s of fp64 numpy oracle work; %d sequence steps "
+                      "in all" % (workers, workers - 1, el, done),
+            "tiny_single_thread": oracle_single_thread_tiny()}
 
 
 # --------------------------------------------------------------------------- main
@@ -353,26 +461,36 @@ def workload_config(cfg: WL.DecodeConfig, world: int) -> dict:
 
 
 def run_reference(args, rank, world):
+    """The oracle as the reference arm, on the host's cores: each step decodes one sequence
+    of the workload in each of `workers` single-threaded processes at once; rank 0 only."""
     cfg = WL.CONFIGS[args.config]
     if rank != 0:
         return
-    inp = oracle_sample(cfg, 0, 1)
-    times = []
-    for i in range(args.warmup + args.steps):
-        rate, done, el = time_oracle(inp, 0.0)
-        if i >= args.warmup:
-            times.append(el)
+    workers = oracle_workers(cfg)
+    times = run_oracle_pool(cfg, 0, workers, steps=args.warmup + args.steps)[args.warmup:]
     ms = 1e3 * sum(times) / len(times)
-    value = 1.0 / (ms * 1e-3)
+    value = workers / (ms * 1e-3)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": dict(workload_config(cfg, 1), step_sample="1 sequence of the workload per step"),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
-                             "sample": "1 of %d sequences per step (full context)" % cfg.B},
+            "config": dict(workload_config(cfg, 1),
+                           step_sample="%d sequences of the workload per step, one per process" % workers),
+            "step_ms_p10_p50_p90": percentiles([1e3 * t for t in times]),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": workers, "kind": "oracle",
+                             "sample": "%d of %d sequences per step (full context), %d single-threaded "
+                                       "processes" % (workers, cfg.B, workers)},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def percentiles(v):
+    """(p10, p50, p90) of a list, nearest-rank."""
+    v = sorted(v)
+    if not v:
+        return None
+    pick = lambda f: v[min(len(v) - 1, max(0, int(math.ceil(f * len(v))) - 1))]
+    return [pick(0.1), pick(0.5), pick(0.9)]
 
 
 def run_gemm(args, rank, world):
@@ -688,108 +806,171 @@ def run_adaptive(args):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    args = parse()
-    if args.config == "layout":
-        return run_layout(args)
-    if args.config == "adaptive":
-        return run_adaptive(args)
-    if args.config == "gemm":
-        rank = int(os.environ.get("RANK", "0"))
-        if rank == 0:
-            run_gemm(args, rank, 1)
-        return
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dist = world > 1
-    if args.impl == "reference":
-        return run_reference(args, rank, world)
-    if args.warmup < 3:
-        args.warmup = 3
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if dist:
-        import datetime
-        import torch.distributed as tdist
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                 device_id=dev)
-    from kv_cache_offload_b200.build import build
-    if rank == 0 or not dist:
-        build()
-    if dist:
-        tdist.barrier()
-    import kv_cache_offload_b200 as dkv
+HEADLINE = "70b_mixed"  # the largest single-GPU decode configuration: the headline line
+HBM_LINE = "8b_hbm"     # the all-HBM configuration, reported beside it in the same run
 
-    cfg = WL.CONFIGS[args.config]
-    if args.batch:
-        import dataclasses
-        cfg = dataclasses.replace(cfg, B=args.batch)
-    wl = Workload(cfg, seed=rank, host_flags=args.host_flags)
-    wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant)
+
+def _nvtx(name):
+    torch.cuda.nvtx.range_push(name)
+
+
+def _nvtx_end():
+    torch.cuda.nvtx.range_pop()
+
+
+def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full: bool, steps: int) -> dict:
+    """Time the decode step of one workload on this rank (every rank makes the same
+    collective calls) and return its JSON fields. `full` adds the end-to-end loop."""
+    import kv_cache_offload_b200 as dkv
+    tdist = None
+    if dist:
+        import torch.distributed as tdist
 
     def barrier():
         if dist:
             tdist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        wl.step()
-    assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
-    if args.profile:
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(args.steps):
-            wl.step()
-        b.record()
-        b.synchronize()
-        assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
-        if rank == 0:
-            print(json.dumps({"profile_run": cfg.name, "B": cfg.B, "attn_splits": wl.splits,
-                              "ms_per_step": a.elapsed_time(b) / args.steps}), flush=True)
-        wl.close()
-        return
-
-    # ---- value: K back-to-back steps, inputs resident in HBM / host tier. The clock
-    # sampler (200 ms period) starts first and the GPU is kept busy with untimed steps for
-    # ~0.6 s so that samples are taken under the same load as the timed region.
-    clocks = ClockSampler(local)
-    barrier()
-    clocks.start()
-    t_end = time.perf_counter() + 0.6
-    while time.perf_counter() < t_end:
-        for _ in range(8):
-            wl.step()
-        torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(args.steps):
-        wl.step()
-    e1.record()
-    barrier()
-    time.sleep(0.25)
-    clk = clocks.stop()
-    t_ms = e0.elapsed_time(e1)
-    assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
-
-    # ---- per-stage durations: the same steps launched serially (no programmatic dependent
-    # launch, so each kernel runs alone), with events between the two launches
-    wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant, serial_launch=1)
-    for _ in range(3):
-        wl.step()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    barrier()
-    for i in range(args.steps):
-        wl.step_timed_stages(evs[i])
-    barrier()
-    stage_ms = [sum(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(args.steps)) / args.steps
-                for k in range(2)]
+    _nvtx("setup " + cfg.name)
+    wl = Workload(cfg, seed=rank, host_flags=args.host_flags)
     wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant)
+    _nvtx_end()
+    try:
+        _nvtx("warmup " + cfg.name)
+        for _ in range(args.warmup):
+            wl.step()
+        assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
+        _nvtx_end()
 
-    # ---- e2e: host buffers in, result out, through the public API. As a serving loop runs
-    # it: step k+1's inputs are copied from pinned host memory on a copy stream into the
-    # second of two device buffer sets while step k computes, and step k's output is read
-    # back on that stream; every copy of every step is inside the timed region.
+        # ---- value: K back-to-back steps, inputs resident in HBM / the host tier. The clock
+        # sampler (200 ms period) starts first and the GPU is kept busy with untimed steps for
+        # ~0.6 s so that samples are taken under the same load as the timed region.
+        clocks = ClockSampler(local)
+        barrier()
+        clocks.start()
+        t_end = time.perf_counter() + 0.6
+        while time.perf_counter() < t_end:
+            for _ in range(8 if wl.kv_host_bytes == 0 else 1):
+                wl.step()
+            torch.cuda.synchronize()
+        _nvtx("timed " + cfg.name)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            wl.step()
+        e1.record()
+        barrier()
+        _nvtx_end()
+        time.sleep(0.25)
+        clk = clocks.stop()
+        t_ms = e0.elapsed_time(e1)
+        assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
+
+        # ---- step-time spread: the same steps with an event after each one (a separate
+        # pass: an event between steps ends the next step's early start)
+        _nvtx("per-step " + cfg.name)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        barrier()
+        evs[0].record()
+        for i in range(steps):
+            wl.step()
+            evs[i + 1].record()
+        barrier()
+        _nvtx_end()
+        per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
+
+        # ---- per-stage durations: the same steps launched serially (no programmatic
+        # dependent launch, so each kernel runs alone), with events between the two launches
+        _nvtx("stages " + cfg.name)
+        wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant, serial_launch=1)
+        for _ in range(3):
+            wl.step()
+        sevs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        barrier()
+        for i in range(steps):
+            wl.step_timed_stages(sevs[i])
+        barrier()
+        stage_ms = [sum(sevs[i][k].elapsed_time(sevs[i][k + 1]) for i in range(steps)) / steps
+                    for k in range(2)]
+        wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant)
+        _nvtx_end()
+
+        e2e_ms, h2d, d2h = 0.0, 0, 0
+        if full:
+            _nvtx("e2e " + cfg.name)
+            e2e_ms, h2d, d2h = time_e2e(wl, steps, barrier)
+            _nvtx_end()
+
+        # ---- max over ranks
+        p10, p50, p90 = percentiles(per_step)
+        vals = reduce_max_over_ranks([t_ms, e2e_ms, p10, p50, p90] + stage_ms, dist, dev)
+        t_ms, e2e_ms, p10, p50, p90 = vals[:5]
+        stage_ms = vals[5:]
+        ms = t_ms / steps
+        value = replica_throughput(cfg.B, world, ms)
+
+        peak, peak_kind = load_peaks()
+        attn_ms = stage_ms[1]
+        achieved = wl.kv_bytes / (attn_ms * 1e-3) / 1e9
+        host_info = None
+        if wl.kv_host_bytes:
+            h2d_peak = measure_h2d_peak(dev)
+            host_gbs = wl.kv_host_bytes / (attn_ms * 1e-3) / 1e9
+            host_info = {"h2d_peak_gbs": h2d_peak, "host_kv_bytes": wl.kv_host_bytes,
+                         "hbm_kv_bytes": wl.kv_hbm_bytes, "achieved_gbs": host_gbs,
+                         "frac": host_gbs / h2d_peak, "link": "PCIe (not NVLink-C2C)",
+                         "host_numa_node": {"gpu_nearest": host_numa_node(dkv, local),
+                                            "host_tier_first_page": dkv.dkv_pool_host_numa_node(wl.pool),
+                                            "policy": "preferred node = the GPU's nearest (DKV_HOST_NUMA_NEAREST)"
+                                            if args.host_flags & 2 else "none"}}
+        tr = profiled_traffic(cfg.name, cfg.B)
+        line = {
+            "value": value, "ms_per_step": ms,
+            "step_ms_p10_p50_p90": [p10, p50, p90],
+            "config": dict(workload_config(cfg, world), attn_splits=wl.splits, attn_variant=args.attn_variant,
+                           attn_kernel_variant=dkv.dkv_decode_attn_variant(wl.pool, cfg.B, wl.lay.max_blocks, cfg.Hq),
+                           l2="inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)),
+            "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
+            # the whole step against the same peak: every byte it must move (cached KV, W, x,
+            # the new K/V rows, out) over the step time (host-tier bytes over the host link)
+            "step_roofline": step_roofline(wl, ms, peak, peak_kind),
+            "stage_ms": {"project": stage_ms[0], "attend_and_combine": stage_ms[1],
+                         "timing": "each kernel alone (serial launches); the step overlaps them"},
+            "roofline": ({"bound": "hbm", "kernel": "attn_splitk_kernel",
+                          "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                          "peak_source": peak_kind, "traffic": tr and tr["bytes"],
+                          "traffic_counter": tr and tr["counter"],
+                          "algorithmic_bytes_per_launch": wl.kv_bytes}
+                         if not wl.kv_host_bytes else
+                         {"bound": "host_link", "kernel": "attn_splitk_kernel",
+                          "achieved": host_info["achieved_gbs"], "peak": host_info["h2d_peak_gbs"], "unit": "GB/s",
+                          "frac": host_info["frac"],
+                          "peak_source": "measured cudaMemcpy H2D (pinned, 1 GiB) in this run",
+                          "traffic": tr and tr["bytes"], "traffic_counter": tr and tr["counter"],
+                          "algorithmic_bytes_per_launch": wl.kv_host_bytes}),
+            "gpu_launches": 2 * steps,
+            "clocks": clk,
+        }
+        if full:
+            line["e2e"] = {"value": replica_throughput(cfg.B, world, e2e_ms / steps), "unit": "tokens/s",
+                           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        if host_info:
+            line["host_link"] = host_info
+            if args.compare_staged:
+                line["staged_swap_baseline"] = run_staged_compare(args, cfg, wl, dev)
+                line["staged_swap_baseline"]["zero_copy_ms"] = ms
+        return line
+    finally:
+        wl.close()
+
+
+def time_e2e(wl, steps, barrier):
+    """The step through the public call with host buffers, as a serving loop runs it: step
+    k+1's inputs are copied from pinned host memory on a copy stream into the second of two
+    device buffer sets while step k computes, and step k's output is read back on that
+    stream; every copy of every step is inside the timed region. Returns (ms for all
+    steps, H2D bytes per step, D2H bytes per step)."""
+    dkv, cfg = wl.dkv, wl.cfg
     xh = wl.x.cpu().pin_memory()
     th, mh, lh = wl.table.cpu().pin_memory(), wl.tmap.cpu().pin_memory(), wl.lens.cpu().pin_memory()
     oh = [torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory() for _ in range(2)]
@@ -814,7 +995,7 @@ def main():
     a.record(main)
     cs.wait_event(a)
     copy_inputs(0)
-    for k in range(args.steps):
+    for k in range(steps):
         i = k % 2
         xd, td, md, ld = ins[i]
         main.wait_event(ev_in[i])
@@ -826,72 +1007,104 @@ def main():
             cs.wait_event(ev_done[1 - i])
             with torch.cuda.stream(cs):
                 oh[1 - i].copy_(outs[1 - i], non_blocking=True)
-        if k + 1 < args.steps:
+        if k + 1 < steps:
             copy_inputs(1 - i)
-    last = (args.steps - 1) % 2
+    last = (steps - 1) % 2
     cs.wait_event(ev_done[last])
     with torch.cuda.stream(cs):
         oh[last].copy_(outs[last], non_blocking=True)
     main.wait_stream(cs)
     b.record(main)
     barrier()
-    e2e_ms = a.elapsed_time(b)
+    return a.elapsed_time(b), h2d, d2h
 
-    # ---- max over ranks
-    vals = reduce_max_over_ranks([t_ms, e2e_ms] + stage_ms, dist, dev)
-    t_ms, e2e_ms = vals[0], vals[1]
-    stage_ms = vals[2:]
-    ms = t_ms / args.steps
-    value = replica_throughput(cfg.B, world, ms)
-    e2e_val = replica_throughput(cfg.B, world, e2e_ms / args.steps)
 
-    peak, peak_kind = load_peaks()
-    attn_ms = stage_ms[1]
-    achieved = wl.kv_bytes / (attn_ms * 1e-3) / 1e9
-    host_info = None
-    if wl.kv_host_bytes:
-        h2d_peak = measure_h2d_peak(dev)
-        host_gbs = wl.kv_host_bytes / (attn_ms * 1e-3) / 1e9
-        host_info = {"h2d_peak_gbs": h2d_peak, "host_kv_bytes": wl.kv_host_bytes,
-                     "achieved_gbs": host_gbs, "frac": host_gbs / h2d_peak,
-                     "link": "PCIe (not NVLink-C2C)"}
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(cfg, world), attn_splits=wl.splits, attn_variant=args.attn_variant,
-                       attn_kernel_variant=dkv.dkv_decode_attn_variant(wl.pool, cfg.B, wl.lay.max_blocks, cfg.Hq),
-                       l2="inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)),
-        "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
-        # the whole step against the same peak: every byte it must move (cached KV, W, x,
-        # the new K/V rows, out) over the step time (host-tier bytes over the host link)
-        "step_roofline": step_roofline(wl, ms, peak, peak_kind),
-        "stage_ms": {"project": stage_ms[0], "attend_and_combine": stage_ms[1],
-                     "timing": "each kernel alone (serial launches); the step overlaps them"},
-        "roofline": ({"bound": "hbm", "kernel": "attn_splitk_kernel",
-                      "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                      "peak_source": peak_kind,
-                      "traffic": profiled_traffic(cfg.name),
-                      "algorithmic_bytes_per_launch": wl.kv_bytes}
-                     if not wl.kv_host_bytes else
-                     {"bound": "host_link", "kernel": "attn_splitk_kernel",
-                      "achieved": host_info["achieved_gbs"], "peak": host_info["h2d_peak_gbs"], "unit": "GB/s",
-                      "frac": host_info["frac"], "peak_source": "measured cudaMemcpy H2D (pinned, 1 GiB) in this run",
-                      "traffic": None, "algorithmic_bytes_per_launch": wl.kv_host_bytes}),
-        "e2e": {"value": e2e_val, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
-        "clocks": clk,
-    }
-    if host_info:
-        line["host_link"] = host_info
-        if args.compare_staged:
-            line["staged_swap_baseline"] = run_staged_compare(args, cfg, wl, dev)
-            line["staged_swap_baseline"]["zero_copy_ms"] = ms
+def host_numa_node(dkv, device_index: int):
+    """The NUMA node the pool's host tier is bound to on this GPU (None where unknown)."""
+    try:
+        n = dkv.dkv_host_numa_node(device_index)
+        return None if n < 0 else n
+    except Exception:
+        return None
+
+
+def main():
+    args = parse()
+    if args.config == "layout":
+        return run_layout(args)
+    if args.config == "adaptive":
+        return run_adaptive(args)
+    if args.config == "gemm":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank == 0:
+            run_gemm(args, rank, 1)
+        return
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = world > 1
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.warmup < 3:
+        args.warmup = 3
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if dist:
+        import datetime
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                 device_id=dev)
+    from kv_cache_offload_b200.build import build
+    if rank == 0 or not dist:
+        build()
+    if dist:
+        tdist.barrier()
+    import kv_cache_offload_b200 as dkv
+
+    cfg = WL.CONFIGS[args.config]
+    if args.batch or args.ctx:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, B=args.batch or cfg.B)
+        if args.ctx:
+            cfg = dataclasses.replace(cfg, ctx=args.ctx, ctx_range=None)
+    if args.profile:
+        wl = Workload(cfg, seed=rank, host_flags=args.host_flags)
+        wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant)
+        for _ in range(args.warmup):
+            wl.step()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            wl.step()
+        b.record()
+        b.synchronize()
+        assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
+        if rank == 0:
+            print(json.dumps({"profile_run": cfg.name, "B": cfg.B, "attn_splits": wl.splits,
+                              "attn_kernel_variant": dkv.dkv_decode_attn_variant(wl.pool, cfg.B, wl.lay.max_blocks,
+                                                                                 cfg.Hq),
+                              "kv_hbm_bytes": wl.kv_hbm_bytes, "kv_host_bytes": wl.kv_host_bytes,
+                              "w_bytes": wl.w_bytes, "ms_per_step": a.elapsed_time(b) / args.steps}), flush=True)
+        wl.close()
+        return
+
+    body = decode_line(cfg, args, world, rank, local, dist, dev, full=True, steps=args.steps)
+    line = {"metric": METRIC, "value": body.pop("value"), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": body.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic"}
+    line.update(body)
+    if args.config == HEADLINE and not args.batch and not args.ctx and not args.no_hbm_line:
+        # the all-HBM layer in the same run: the HBM-roofline bar beside the host-link one
+        torch.cuda.empty_cache()
+        hsteps = max(args.steps, 100)  # 0.4 ms steps: more of them for a stable mean
+        hl = decode_line(WL.CONFIGS[HBM_LINE], args, world, rank, local, dist, dev, full=False, steps=hsteps)
+        hl.update(unit="tokens/s", steps=hsteps)
+        line["hbm_line"] = hl
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, 0, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    wl.close()
     if dist:
         tdist.barrier()
         tdist.destroy_process_group()

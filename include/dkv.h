@@ -44,6 +44,8 @@ extern "C" {
 #define DKV_ERR_BAD_TABLE   (-5)  /* device-side table validation failed (dkv_check) */
 #define DKV_ERR_TIMEOUT     (-6)  /* a bounded device-side wait gave up (dkv_check) */
 #define DKV_ERR_CAPACITY    (-7)  /* request exceeds a fixed capacity */
+#define DKV_ERR_INTERNAL    (-8)  /* a range check of the debug build (libdkv_debug.so, built
+                                     with DKV_DEBUG) failed inside a kernel (dkv_check) */
 
 #define DKV_TIER_HBM  0
 #define DKV_TIER_HOST 1
@@ -52,6 +54,8 @@ extern "C" {
 #define DKV_LAYOUT_PAGE_FIRST  1  /* tier = [P][L][2][Hkv][T][D] */
 
 #define DKV_HOST_WRITE_COMBINED 1 /* host tier allocated write-combined */
+#define DKV_HOST_NUMA_NEAREST   2 /* host tier placed on the NUMA node nearest the pool's GPU
+                                     (see dkv_host_numa_node) */
 
 typedef struct dkv_pool dkv_pool;  /* opaque; owned by the library */
 
@@ -71,7 +75,7 @@ typedef struct dkv_pool_config {
   int64_t hbm_blocks;    /* physical blocks in the HBM tier (>= 0) */
   int64_t host_blocks;   /* physical blocks in the host tier (>= 0) */
   int32_t layout;        /* DKV_LAYOUT_* */
-  int32_t host_flags;    /* 0 or DKV_HOST_WRITE_COMBINED */
+  int32_t host_flags;    /* DKV_HOST_* bits (0: write-back pages, no NUMA preference) */
   void*   hbm_base;      /* optional caller-owned device buffer of at least the HBM tier's
                             size (256-byte aligned); NULL = the library allocates it */
 } dkv_pool_config;
@@ -81,21 +85,37 @@ typedef struct dkv_tuning {
   int32_t attn_splits;   /* split-K factor of the attention grid (per sequence, kv head) */
   int32_t proj_splits;   /* cluster size of the projection (its reduction split), <= 16 */
   int32_t attn_variant;  /* attention kernel: 0 automatic (see dkv_decode_attn_variant),
-                            5 CUDA-core products (q in registers, 3 consumer warps,
-                            6-stage ring, 4 CTAs/SM; G = 8 runs the variant-1 shape),
-                            1 CUDA cores with 4 consumer warps, an 8-stage ring and
-                            3 CTAs/SM, 2 CUDA cores with q in
-                            shared memory (4-stage ring, 4 CTAs/SM), 6 tensor-core
-                            products (4-stage ring, 4 CTAs/SM), 7 tensor cores with an
-                            8-stage ring (3 CTAs/SM); other values are invalid. The
-                            tensor-core consumers are opt-in: the design reserves the
-                            tensor cores for the projection */
-  int32_t attn_lsu_hbm;  /* 1: load HBM-tier blocks with 16-byte cp.async, not bulk copies */
+                            5 CUDA-core products with q in registers, three consumer slots
+                            and a 6-stage ring (G <= 4: one warp per slot, 4 CTAs/SM;
+                            G = 8: two warps per slot, 2 CTAs/SM), 1 CUDA cores with four
+                            slots and an 8-stage ring (3 CTAs/SM; G = 8: two warps per
+                            slot, 1 CTA/SM), 8 (G = 8 only, else as 1) two slots of two
+                            warps, a 4-stage ring, 3 CTAs/SM, 6 tensor-core products
+                            (4-stage ring, 4 CTAs/SM), 7 tensor cores with an 8-stage
+                            ring (3 CTAs/SM); other values are invalid. The tensor-core
+                            consumers are opt-in: the design reserves the tensor cores
+                            for the projection */
+  int32_t attn_lsu_hbm;  /* load paths of the CUDA-core attention, bits: 1 = HBM-tier blocks
+                            by 16-byte cp.async instead of bulk copies (TMA engine); 2 =
+                            host-tier blocks by bulk copies from the mapped host memory
+                            instead of 16-byte cp.async from all 32 lanes of the producer */
   int32_t serial_launch; /* 1: launch the decode kernels without programmatic dependent
                             launch (each starts when the one before has finished: for
                             timing the kernels one by one, or when Wqkv is written by the
-                            kernel directly ahead); 0: overlap their boundaries */
-  int32_t reserved[3];
+                            kernel directly ahead); 2: overlap only inside a step (the
+                            attention streams cached KV while the projection finishes; the
+                            kernel after the attention starts when it has finished);
+                            0: overlap both boundaries (the attention also lets the next
+                            kernel, e.g. the next step's projection, start early) */
+  int32_t wait_limit_us; /* limit of each bounded wait inside the attention kernel, in
+                            microseconds (0 = 4 s). On giving up a wait the kernel sets
+                            DKV_ERR_TIMEOUT in the pool's status word and returns */
+  int32_t test_withhold_block; /* test hook of the bounded waits: 1 = the attention's first
+                            CTA (split 0, kv head 0, sequence 0) never loads its first block
+                            nor signals its stage, so that stage's consumer gives up after
+                            wait_limit_us (output of that (sequence, kv head) is then
+                            undefined, dkv_check reports DKV_ERR_TIMEOUT); 0 = off */
+  int32_t reserved[1];
 } dkv_tuning;
 
 /*
@@ -107,6 +127,24 @@ typedef struct dkv_tuning {
  * Tier contents are uninitialised.
  */
 int dkv_pool_create(const dkv_pool_config* cfg, dkv_pool** out);
+
+/*
+ * NUMA placement of the host tier. GPUs of one host each read their own host tier over
+ * their own PCIe link but share the host's memory (DirectKV leaves several GPUs sharing
+ * CPU memory as future work: "长上下文 LLM 的零拷贝 KV Cache 卸载（OSDI 2026）", 局限与后续
+ * 工作). With DKV_HOST_NUMA_NEAREST the pool allocates its host tier under a "preferred"
+ * memory policy for the node its GPU's PCIe device reports, restoring the calling thread's
+ * policy afterwards (a full node falls back to others; no error).
+ *  - dkv_numa_node_of_pci: the node sysfs gives for a PCI device: reads
+ *    <sysfs_root>/bus/pci/devices/<bus id, lower case, 4-digit domain>/numa_node
+ *    (sysfs_root NULL = "/sys"); -1 when absent or negative (no NUMA information).
+ *  - dkv_host_numa_node: the same for a CUDA device (its cudaDeviceGetPCIBusId); -1 if none.
+ *  - dkv_pool_host_numa_node: the node that actually backs the first page of the pool's
+ *    host tier (-1 without a host tier or when the kernel does not say), or DKV_ERR_ARG.
+ */
+int dkv_numa_node_of_pci(const char* sysfs_root, const char* pci_bus_id);
+int dkv_host_numa_node(int device);
+int dkv_pool_host_numa_node(const dkv_pool* pool);
 
 /* Free both tiers (not a caller-supplied hbm_base) and the pool. Synchronises the device. */
 int dkv_pool_destroy(dkv_pool* pool);
@@ -225,7 +263,12 @@ int dkv_decode_combine(dkv_pool* pool, int B, int max_blocks, int hidden, int nu
  * which every GPU that loads the library holds until the process exits. The call allocates
  * nothing (no cudaMalloc/cudaFree, no allocating library routine).
  *  - The first call on a device looks up that device's array address (cudaGetSymbolAddress
- *    with the device current); make that first call before any stream capture.
+ *    with the device current); make that first call before any stream capture. Under CUDA's
+ *    lazy module loading (the default) the array's 16 MiB of device memory are committed at
+ *    that first call, so a caller that reserves the rest of the device's memory up front
+ *    makes one call first. The pool's device must be current (else DKV_ERR_ARG).
+ *  - Shape errors return the same codes as dkv_decode_step (e.g. DKV_ERR_UNSUPPORTED for
+ *    B > 32).
  *  - Shapes whose workspace (dkv_decode_workspace_bytes) exceeds the capacity are rejected
  *    with DKV_ERR_CAPACITY and nothing is launched.
  *  - Every call shares the one array per device and it keeps the last call's contents;
@@ -272,8 +315,10 @@ int dkv_convert_layout(dkv_pool* pool, int tier, void* dst, size_t dst_bytes, vo
  *   Bt[N][K] (bf16; Bt[n][k] = B[k][n]) in mapped pinned host memory (pass its device
  *   alias) or, for DKV_GEMM_DEVICE, in device memory.
  * Variants:
- *   DKV_GEMM_CPU_AWARE        B-panel-major tile order: each B tile crosses the host link
- *                             once and is reused from L2; A is re-read from HBM per panel.
+ *   DKV_GEMM_CPU_AWARE        B-panel-major tile order: each B column panel is copied
+ *                             from host memory into a rotating HBM panel buffer (inside the
+ *                             workspace) exactly once and read from there, so each B tile
+ *                             crosses the host link once; A is re-read from HBM per panel.
  *   DKV_GEMM_NAIVE_ZERO_COPY  row-major tile order: B re-read over the host link by every
  *                             128-row tile row of C.
  *   DKV_GEMM_STAGED_SWAP      cudaMemcpyAsync of all of B into the workspace ("swap" into a
@@ -305,7 +350,9 @@ int dkv_gemm(int variant, const uint16_t* A, const uint16_t* Bt, float* C, int M
 /*
  * Synchronise `stream`, then read and clear the pool's device status word.
  * Returns DKV_OK, DKV_ERR_BAD_TABLE (a kernel skipped a block with a bad tier or physical
- * id, or a context exceeding max_blocks*T), DKV_ERR_TIMEOUT, or DKV_ERR_CUDA.
+ * id, or a context exceeding max_blocks*T), DKV_ERR_TIMEOUT, DKV_ERR_INTERNAL (debug build
+ * only: a kernel's computed block, slot or workspace index fell outside its buffer; the
+ * access was skipped), or DKV_ERR_CUDA.
  */
 int dkv_check(dkv_pool* pool, void* stream);
 

@@ -13,7 +13,8 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libdkv.so")
+# DKV_LIBRARY=debug selects the build with device-side range checks (libdkv_debug.so)
+LIB_PATH = os.path.join(_HERE, "libdkv_debug.so" if os.environ.get("DKV_LIBRARY") == "debug" else "libdkv.so")
 INCLUDE = os.path.join(os.path.dirname(_HERE), "include")
 HEADER = os.path.join(INCLUDE, "dkv.h")
 
@@ -25,12 +26,14 @@ DKV_ERR_UNSUPPORTED = -4
 DKV_ERR_BAD_TABLE = -5
 DKV_ERR_TIMEOUT = -6
 DKV_ERR_CAPACITY = -7
+DKV_ERR_INTERNAL = -8
 
 DKV_TIER_HBM = 0
 DKV_TIER_HOST = 1
 DKV_LAYOUT_LAYER_FIRST = 0
 DKV_LAYOUT_PAGE_FIRST = 1
 DKV_HOST_WRITE_COMBINED = 1
+DKV_HOST_NUMA_NEAREST = 2
 DKV_COPY_DMA = 0
 DKV_COPY_KERNEL = 1
 DKV_GEMM_CPU_AWARE = 0
@@ -58,7 +61,8 @@ class dkv_pool_config(ctypes.Structure):
 class dkv_tuning(ctypes.Structure):
     _fields_ = [("attn_splits", ctypes.c_int32), ("proj_splits", ctypes.c_int32),
                 ("attn_variant", ctypes.c_int32), ("attn_lsu_hbm", ctypes.c_int32),
-                ("serial_launch", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("serial_launch", ctypes.c_int32), ("wait_limit_us", ctypes.c_int32),
+                ("test_withhold_block", ctypes.c_int32), ("reserved", ctypes.c_int32 * 1)]
 
 
 class dkv_bm_config(ctypes.Structure):
@@ -119,6 +123,9 @@ _SIGS = {
                                      _I, _I, _F, _P, _SZ, ctypes.POINTER(_P)]),
     "dkv_graph_launch": (_I, [_P, _P]),
     "dkv_graph_destroy": (_I, [_P]),
+    "dkv_numa_node_of_pci": (_I, [ctypes.c_char_p, ctypes.c_char_p]),
+    "dkv_host_numa_node": (_I, [_I]),
+    "dkv_pool_host_numa_node": (_I, [_P]),
     "dkv_last_error": (ctypes.c_char_p, []),
     "dkv_version": (ctypes.c_char_p, []),
 }
@@ -217,9 +224,29 @@ def dkv_pool_tier_ptr(pool: int, tier: int):
 
 
 def dkv_pool_set_tuning(pool: int, attn_splits: int = 0, proj_splits: int = 0,
-                        attn_variant: int = 0, attn_lsu_hbm: int = 0, serial_launch: int = 0):
-    t = dkv_tuning(attn_splits, proj_splits, attn_variant, attn_lsu_hbm, serial_launch)
+                        attn_variant: int = 0, attn_lsu_hbm: int = 0, serial_launch: int = 0,
+                        wait_limit_us: int = 0, test_withhold_block: int = 0):
+    t = dkv_tuning(attn_splits, proj_splits, attn_variant, attn_lsu_hbm, serial_launch, wait_limit_us,
+                   test_withhold_block)
     _chk(lib().dkv_pool_set_tuning(pool, ctypes.byref(t)))
+
+
+def dkv_numa_node_of_pci(sysfs_root: Optional[str], pci_bus_id: str) -> int:
+    """NUMA node sysfs reports for a PCI device (-1 if none)."""
+    return lib().dkv_numa_node_of_pci(None if sysfs_root is None else sysfs_root.encode(), pci_bus_id.encode())
+
+
+def dkv_host_numa_node(device: int) -> int:
+    """NUMA node nearest CUDA device `device` (-1 if the platform reports none)."""
+    return lib().dkv_host_numa_node(device)
+
+
+def dkv_pool_host_numa_node(pool: int) -> int:
+    """Node backing the first page of the pool's host tier (-1 if unknown or no host tier)."""
+    r = lib().dkv_pool_host_numa_node(pool)
+    if r < -1:
+        raise DkvError(r, dkv_last_error())
+    return r
 
 
 def host_tier_tensor(pool: int) -> torch.Tensor:

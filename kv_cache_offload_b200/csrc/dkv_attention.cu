@@ -21,8 +21,8 @@
 // Scores are in the log2 domain: q arrives pre-scaled by log2(e)/sqrt(D), so p = 2^(s - m).
 // Two consumer implementations:
 //  * CUDA cores (the default = variant 5: three slots, a 6-stage ring, four CTAs per SM;
-//    variant 1: four slots, an 8-stage ring, three CTAs per SM; variant 2 keeps q in
-//    shared memory): packed fp32x2 FMAs. A decode query group is G <= 8 rows, G flops per KV byte: an HBM-bound
+//    variant 1: four slots, an 8-stage ring, three CTAs per SM; at G = 8 a slot is two
+//    warps of four heads each): packed fp32x2 FMAs. A decode query group is G <= 8 rows, G flops per KV byte: an HBM-bound
 //    product, not a dense contraction, and the tensor cores are kept for the projection.
 //  * tensor cores (opt-in, variants 6 and 7): per block, S = Q.K^T and O^T += V^T.P^T as
 //    m16n8k16 bf16 mma.sync with fp32 accumulation. The G query rows of a kv head are padded to the
@@ -58,7 +58,7 @@ struct AttnCfg {
   static constexpr int DPL = D / 32;   // value dims per lane in P.V
   static constexpr int QCH = D / 64;   // 16-byte key chunks per lane per token in Q.K
   static constexpr int NV = HPW * 4;   // partial scores per lane (heads x 4 tokens)
-  static constexpr int LOGH = HPW == 4 ? 2 : (HPW == 2 ? 1 : 0);
+  static constexpr int LOGH = HPW == 8 ? 3 : (HPW == 4 ? 2 : (HPW == 2 ? 1 : 0));
   static constexpr int LOWMASK = (1 << (3 - LOGH)) - 1;  // dg bits shared by one head
   static constexpr int NR = NV >= 8 ? NV / 8 : 1;        // scores per lane after reduction
   static constexpr int OFF_P = NST * STAGE_BYTES;
@@ -198,6 +198,7 @@ __device__ __forceinline__ void attn_merge_combine(const AttnParams& p, uint8_t*
       }
     }
     const int64_t base = ((int64_t)b * p.Hq + g * G + hh) * p.S + s;
+    if (!DKV_DEBUG_RANGE(pool.status, base, base + 1, (int64_t)gridDim.z * p.Hq * p.S)) continue;
     p.part_acc[base * D + d] = A;
     if (d == 0) p.part_ml[base] = make_float2(M, Ls);
   }
@@ -215,6 +216,9 @@ __device__ __forceinline__ void attn_merge_combine(const AttnParams& p, uint8_t*
       const float* kn = p.knew + ((int64_t)b * pool.Hkv + g) * D;
       for (int hh = warp; hh < G; hh += NCW) {
         const int hg = g * G + hh;
+        if (!DKV_DEBUG_RANGE(pool.status, (int64_t)b * p.Hq + hg, (int64_t)b * p.Hq + hg + 1,
+                             (int64_t)gridDim.z * p.Hq))
+          continue;
         const float sn = new_token_score(p.qs + ((int64_t)b * p.Hq + hg) * D, kn, D, lane);
         combine_head_warp<D>(p.part_ml, p.part_acc, p.S, ((int64_t)b * p.Hq + hg) * p.S, 1, sn,
                              p.vnew + ((int64_t)b * pool.Hkv + g) * D, p.out + ((int64_t)b * p.Hq + hg) * D, lane);
@@ -233,8 +237,9 @@ __device__ __forceinline__ void attn_merge_combine(const AttnParams& p, uint8_t*
 //     the 16-byte piece c of row r stored at piece c ^ (r mod 8) (the TMA 128-byte
 //     swizzle; the stage is 1024-byte aligned); HBM blocks arrive by 2*D/64 TMA tensor
 //     copies through `tmap` (the HBM tier as [rows][D]).
-// Host-tier blocks (and HBM blocks when p.lsu_hbm) arrive by 16-byte cp.async from all 32
-// lanes into the same layout. Table entries are fetched 32 blocks at a time (lane l holds
+// Host-tier blocks (and HBM blocks when bit 0 of p.lsu_hbm is set) arrive by 16-byte
+// cp.async from all 32 lanes into the same layout; with bit 1 set, host blocks of the packed
+// layout arrive by bulk copies from the mapped host memory instead. Table entries are fetched 32 blocks at a time (lane l holds
 // block base + l) and broadcast by shuffle, so no dependent global load sits on the
 // per-block path.
 template <int D, int NST, bool SW>
@@ -255,6 +260,8 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
   const uint16_t* kbase1 = pool.tier[1] + chunk_offset(pool, 1, p.layer, 0, 0, g);
   int pf_tier = 0, pf_phys = 0;
   int issued = 0;
+  // test hook (bounded-wait test): the first CTA never loads nor signals its first block
+  const int withheld = (p.withhold && blockIdx.x == 0 && g == 0 && b == 0) ? 0 : -1;
   for (int i = 0; i < n_local; ++i) {
     if ((i & 31) == 0) {
       const int j = j0 + i + lane;
@@ -265,7 +272,11 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
     }
     const int st = i % NST;
     const int k = i / NST;
-    if (k > 0 && !mbar_wait_bounded(&empty[st], (k - 1) & 1, pool.status)) break;
+    if (k > 0 && !mbar_wait_bounded(&empty[st], (k - 1) & 1, pool.status, p.wait_ns)) break;
+    if (i == withheld) {
+      issued = i + 1;
+      continue;
+    }
     const int j = j0 + i;
     const int tier = __shfl_sync(0xffffffffu, pf_tier, i & 31);
     const int64_t phys = __shfl_sync(0xffffffffu, pf_phys, i & 31);
@@ -279,6 +290,13 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
       if (lane == 0) flag_error(pool.status, kErrBadBlock);
     }
     uint8_t* dst = stages + st * DATA_BYTES;
+    const uint16_t* kp = (tier ? kbase1 : kbase0) + phys * pstride;
+    const uint16_t* vp = kp + kvoff;
+    if (valid) {  // the K and V chunks lie inside the tier (DKV_DEBUG build)
+      const int64_t ko = kp - tier_base(pool, tier), vo = vp - tier_base(pool, tier);
+      valid = DKV_DEBUG_RANGE(pool.status, ko, ko + TD, tier_elems(pool, tier)) &&
+              DKV_DEBUG_RANGE(pool.status, vo, vo + TD, tier_elems(pool, tier));
+    }
     if (lane == 0) flags[st] = valid ? ntok : -1;
     if (!valid) {
       mbar_arrive(&full[st]);
@@ -286,9 +304,9 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
       issued = i + 1;
       continue;
     }
-    const uint16_t* kp = (tier ? kbase1 : kbase0) + phys * pstride;
-    const uint16_t* vp = kp + kvoff;
-    if (tier == DKV_TIER_HBM && !p.lsu_hbm) {
+    // bulk copies (TMA engine) for HBM blocks, and for host blocks when asked (the swizzled
+    // stage layout takes HBM tensor-map copies only)
+    if ((tier == DKV_TIER_HBM && !(p.lsu_hbm & 1)) || (!SW && tier == DKV_TIER_HOST && (p.lsu_hbm & 2))) {
       if (lane == 0) {
         mbar_arrive_expect_tx(&full[st], DATA_BYTES);
         mbar_arrive(&full[st]);
@@ -327,15 +345,37 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
   // issued loads are the only ones that can be in flight; their stage barrier is at the
   // load's phase or past it, so the parity wait is exact (bounded, 100 ms).
   for (int j = issued > NST ? issued - NST : 0; j < issued; ++j)
-    mbar_wait_bounded(&full[j % NST], (j / NST) & 1, pool.status, 100000000ull);
+    if (j != withheld)
+      mbar_wait_bounded(&full[j % NST], (j / NST) & 1, pool.status, p.wait_ns < 100000000ull ? p.wait_ns : 100000000ull);
 }
 
-// QS: keep q in shared memory instead of registers (fewer registers, more CTAs per SM).
-template <int D, int HPW, int WPB, int NST, int MINB, bool QS, int SL>
+// Longest sequences first. CTAs start in grid order, so the z index of the grid is mapped
+// to sequences by decreasing cached length (ties by index): the CTAs of the longest
+// sequences take the first slots and the short ones fill in behind them, so a ragged batch
+// finishes together (a uniform batch keeps its order). Warp 0 ranks the B <= 32 lengths.
+__device__ __forceinline__ int longest_first_sequence(const AttnParams& p, int* s_b, int warp, int lane) {
+  if (warp == 0) {
+    const int nB = (int)gridDim.z;
+    const int len = lane < nB ? __ldcg(p.seq_lens + lane) : INT32_MIN;
+    int rank = 0;
+    for (int j = 0; j < nB; ++j) {
+      const int lj = __shfl_sync(0xffffffffu, len, j);
+      rank += (lj > len) || (lj == len && j < lane);
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, lane < nB && rank == (int)blockIdx.z);
+    if (lane == 0) *s_b = m ? __ffs(m) - 1 : (int)blockIdx.z;
+  }
+  __syncthreads();
+  return *s_b;
+}
+
+// QSM: q in shared memory instead of registers (the group-of-8 shape with one warp per
+// block, whose eight heads of q would not fit in registers).
+template <int D, int HPW, int WPB, int NST, int MINB, int SL, bool QSM>
 __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
     attn_splitk_kernel(const AttnParams p) {
   using C = AttnCfg<D, HPW, WPB, NST, SL>;
-  constexpr int OFF_Q = (C::SMEM + 15) / 16 * 16;  // q area (QS only): [G][QCH][2][8][4] fp32
+  constexpr int OFF_Q = (C::SMEM + 15) / 16 * 16;  // q area (QSM only): [G][QCH][2][8][4] fp32
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* stages = reinterpret_cast<uint16_t*>(smem);
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
@@ -344,14 +384,15 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
   uint64_t* empty = full + NST;
 
-  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int s_b;
+  const int s = blockIdx.x, g = blockIdx.y, b = longest_first_sequence(p, &s_b, warp, lane);
   const PoolView& pool = p.pool;
   // Behind this step's projection (p.early_kv) only the consumers wait for it, before q;
   // the producer streams the cached blocks at once (see attn_mma_kernel for why that is
   // safe). Behind anything else every thread waits first.
   if (!p.early_kv) griddep_wait();
-  if (threadIdx.x == 0) griddep_launch_dependents();
+  if (p.signal_next && threadIdx.x == 0) griddep_launch_dependents();
 
   // cached tokens of this sequence, clamped to what the table can hold
   int ctx = __ldcg(p.seq_lens + b);
@@ -386,11 +427,11 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
   const int hbase = g * C::G + hq * HPW;  // first global q head of this warp
 
   // q of this lane's key dims, as (even, odd) dim pairs for the packed fp32x2 FMA: in
-  // registers, or (QS) in shared memory laid out [head][hh][half][dg][4] so that the eight
-  // dg lanes read 128 contiguous bytes.
-  float2 q2[QS ? 1 : HPW][QS ? 1 : C::QCH][4];
+  // registers, or (QSM) in shared memory laid out [head][hh][half][dg][4] so that the
+  // eight dg lanes read 128 contiguous bytes
+  float2 q2[QSM ? 1 : HPW][QSM ? 1 : C::QCH][4];
   float* qsm = reinterpret_cast<float*>(smem + OFF_Q);
-  if constexpr (QS) {
+  if constexpr (QSM) {
     for (int e = threadIdx.x; e < C::G * D; e += C::NCW * 32) {
       const int h = e / D, d = e % D, c = d / 8, w = d % 8;
       qsm[(((h * C::QCH + c / 8) * 2 + w / 4) * 8 + c % 8) * 4 + w % 4] =
@@ -426,7 +467,7 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
 
   for (int i = slot; i < n_local; i += SL) {
     const int st = i % NST;
-    if (!mbar_wait_bounded(&full[st], (i / NST) & 1, pool.status)) break;
+    if (!mbar_wait_bounded(&full[st], (i / NST) & 1, pool.status, p.wait_ns)) break;
     const int ntok = flags[st];
     if (ntok > 0) {
       const uint16_t* Ks = stages + st * C::STAGE_ELEMS;
@@ -437,7 +478,9 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
       float2 v2[C::NV];
 #pragma unroll
       for (int x = 0; x < C::NV; ++x) v2[x] = make_float2(0.f, 0.f);
-      if constexpr (QS) {
+      if constexpr (QSM) {
+        // per 16-byte key chunk: the lane's four tokens unpacked once, then every head's q
+        // read from shared memory (broadcast across the four token groups)
 #pragma unroll
         for (int hh = 0; hh < C::QCH; ++hh) {
           float2 kk[4][4];
@@ -468,26 +511,26 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
         }
       } else {
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) {
-          const int t = tg + 4 * i4;
+      for (int i4 = 0; i4 < 4; ++i4) {
+        const int t = tg + 4 * i4;
 #pragma unroll
-          for (int hh = 0; hh < C::QCH; ++hh) {
-            const uint4 w = *reinterpret_cast<const uint4*>(Ks + t * D + (dg + 8 * hh) * 8);
-            const float2 k0 = make_float2(bf16lo(w.x), bf16hi(w.x));
-            const float2 k1 = make_float2(bf16lo(w.y), bf16hi(w.y));
-            const float2 k2 = make_float2(bf16lo(w.z), bf16hi(w.z));
-            const float2 k3 = make_float2(bf16lo(w.w), bf16hi(w.w));
+        for (int hh = 0; hh < C::QCH; ++hh) {
+          const uint4 w = *reinterpret_cast<const uint4*>(Ks + t * D + (dg + 8 * hh) * 8);
+          const float2 k0 = make_float2(bf16lo(w.x), bf16hi(w.x));
+          const float2 k1 = make_float2(bf16lo(w.y), bf16hi(w.y));
+          const float2 k2 = make_float2(bf16lo(w.z), bf16hi(w.z));
+          const float2 k3 = make_float2(bf16lo(w.w), bf16hi(w.w));
 #pragma unroll
-            for (int h = 0; h < HPW; ++h) {
-              float2 a = v2[h * 4 + i4];
-              a = __ffma2_rn(q2[h][hh][0], k0, a);
-              a = __ffma2_rn(q2[h][hh][1], k1, a);
-              a = __ffma2_rn(q2[h][hh][2], k2, a);
-              a = __ffma2_rn(q2[h][hh][3], k3, a);
-              v2[h * 4 + i4] = a;
-            }
+          for (int h = 0; h < HPW; ++h) {
+            float2 a = v2[h * 4 + i4];
+            a = __ffma2_rn(q2[h][hh][0], k0, a);
+            a = __ffma2_rn(q2[h][hh][1], k1, a);
+            a = __ffma2_rn(q2[h][hh][2], k2, a);
+            a = __ffma2_rn(q2[h][hh][3], k3, a);
+            v2[h * 4 + i4] = a;
           }
         }
+      }
       }
       float v[C::NV];
 #pragma unroll
@@ -661,8 +704,9 @@ __global__ void __launch_bounds__((kSlots + 1) * 32, MINB)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BARS);
   uint64_t* empty = full + NST;
 
-  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int s_b;
+  const int s = blockIdx.x, g = blockIdx.y, b = longest_first_sequence(p, &s_b, warp, lane);
   const PoolView& pool = p.pool;
   // Launched with programmatic dependent launch behind the projection of the same step
   // (p.early_kv): q, the new token's k/v and the split counters come from it, so the
@@ -672,7 +716,7 @@ __global__ void __launch_bounds__((kSlots + 1) * 32, MINB)
   // producer starts at once; tables and positions are read through L2. Launched behind
   // anything else, every thread waits first.
   if (!p.early_kv) griddep_wait();
-  if (threadIdx.x == 0) griddep_launch_dependents();
+  if (p.signal_next && threadIdx.x == 0) griddep_launch_dependents();
 
   int ctx = __ldcg(p.seq_lens + b);
   if (ctx < 0 || ctx / kT + 1 > p.max_blocks) {
@@ -742,7 +786,7 @@ __global__ void __launch_bounds__((kSlots + 1) * 32, MINB)
   for (int i = slot; i < n_local; i += kSlots) {
     const int st = i % NST;
     // warp-uniform: a give-up on any lane ends the loop for the whole warp
-    if (!__all_sync(FULL, mbar_wait_bounded(&full[st], (i / NST) & 1, pool.status))) break;
+    if (!__all_sync(FULL, mbar_wait_bounded(&full[st], (i / NST) & 1, pool.status, p.wait_ns))) break;
     const int ntok = flags[st];
     if (ntok > 0) {
       const uint32_t kb = sbase + st * STAGE;
@@ -898,11 +942,11 @@ static int launch_pdl(void (*fn)(KArgs...), dim3 grid, int threads, int smem, cu
   return cuda_check(cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...), "attention launch");
 }
 
-template <int D, int HPW, int WPB, int NST, int MINB, bool QS = false, int SL = kSlots>
+template <int D, int HPW, int WPB, int NST, int MINB, int SL = kSlots, bool QSM = false>
 static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
   using C = AttnCfg<D, HPW, WPB, NST, SL>;
-  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB, QS, SL>;
-  constexpr int smem = QS ? (C::SMEM + 15) / 16 * 16 + C::G * D * 4 : C::SMEM;
+  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB, SL, QSM>;
+  constexpr int smem = QSM ? (C::SMEM + 15) / 16 * 16 + C::G * D * 4 : C::SMEM;
   static bool attr_done = false;  // per instantiation
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -967,20 +1011,14 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
   }
   if (variant == 5 || variant == 0) {
     switch (G) {
-      case 1: return launch_attn_t<D, 1, 1, 6, 4, false, 3>(p, B, Hkv, st);
-      case 2: return launch_attn_t<D, 2, 1, 6, 4, false, 3>(p, B, Hkv, st);
-      case 4: return launch_attn_t<D, 4, 1, 6, 4, false, 3>(p, B, Hkv, st);
-      default: break;  // G = 8: the variant-1 shape
+      case 1: return launch_attn_t<D, 1, 1, 6, 4, 3>(p, B, Hkv, st);
+      case 2: return launch_attn_t<D, 2, 1, 6, 4, 3>(p, B, Hkv, st);
+      case 4: return launch_attn_t<D, 4, 1, 6, 4, 3>(p, B, Hkv, st);
+      case 8: return launch_attn_t<D, 4, 2, 6, 2, 3>(p, B, Hkv, st);
     }
   }
-  if (variant == 2) {
-    switch (G) {
-      case 1: return launch_attn_t<D, 1, 1, 4, 4, true>(p, B, Hkv, st);
-      case 2: return launch_attn_t<D, 2, 1, 4, 4, true>(p, B, Hkv, st);
-      case 4: return launch_attn_t<D, 4, 1, 4, 4, true>(p, B, Hkv, st);
-      default: break;  // G = 8: the variant-1 shape
-    }
-  }
+  if (variant == 8 && G == 8) return launch_attn_t<D, 4, 2, 4, 3, 2>(p, B, Hkv, st);
+  if (variant == 9 && G == 8) return launch_attn_t<D, 8, 1, 6, 3, 3, true>(p, B, Hkv, st);
   switch (G) {
     case 1: return launch_attn_t<D, 1, 1, 8, 3>(p, B, Hkv, st);
     case 2: return launch_attn_t<D, 2, 1, 8, 3>(p, B, Hkv, st);
@@ -993,7 +1031,8 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
 int attention_ctas_per_sm(int G, int variant) {
   if (variant == 6) return G == 8 ? 2 : 4;
   if (variant == 7) return G == 8 ? 2 : 3;
-  if (variant == 2 || variant == 5 || variant == 0) return G == 8 ? 1 : 4;
+  if ((variant == 8 || variant == 9) && G == 8) return 3;
+  if (variant == 5 || variant == 0) return G == 8 ? 2 : 4;
   return G == 8 ? 1 : 3;
 }
 

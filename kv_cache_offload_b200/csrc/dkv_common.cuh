@@ -17,6 +17,7 @@ enum : int {
   kErrCtxTooLong = 4,
   kErrTimeout = 8,
   kErrBadPlan = 16,
+  kErrDebugBounds = 32,  // a DKV_DEBUG range check failed (an indexing bug, not bad input)
 };
 
 // What a kernel needs to address the pool.
@@ -51,6 +52,26 @@ __host__ __device__ __forceinline__ int64_t tier_blocks(const PoolView& p, int t
 __device__ __forceinline__ void flag_error(int* status, int bits) {
   if (status) atomicOr(status, bits);
 }
+
+// Elements of a tier (every layer, K and V, every kv head, T tokens of D).
+__host__ __device__ __forceinline__ int64_t tier_elems(const PoolView& p, int tier) {
+  return tier_blocks(p, tier) * p.L * 2 * p.Hkv * p.T * p.D;
+}
+
+// Range checks of the DKV_DEBUG build: every block, slot and workspace access whose index
+// the kernel computed is checked to lie in its buffer ([lo, hi) within [0, n)); a failing
+// access is skipped and flags kErrDebugBounds (dkv_check: DKV_ERR_INTERNAL). The release
+// build compiles them to `true`.
+#ifdef DKV_DEBUG
+__device__ __forceinline__ bool debug_in_range(int* status, int64_t lo, int64_t hi, int64_t n) {
+  if (lo >= 0 && lo <= hi && hi <= n) return true;
+  flag_error(status, kErrDebugBounds);
+  return false;
+}
+#define DKV_DEBUG_RANGE(status, lo, hi, n) ::dkv::debug_in_range((status), (lo), (hi), (n))
+#else
+#define DKV_DEBUG_RANGE(status, lo, hi, n) true
+#endif
 
 // ---------------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start before the kernel

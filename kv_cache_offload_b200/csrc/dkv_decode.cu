@@ -145,7 +145,7 @@ int dkv_decode_project(dkv_pool* pool, int layer, const uint16_t* x, const uint1
   a.vnew = reinterpret_cast<float*>(ws + w.off_vnew);
   a.attn_cnt = reinterpret_cast<int*>(ws + w.off_cnt);
   a.cluster = pool->tuning.proj_splits;
-  a.pdl = !pool->tuning.serial_launch;
+  a.pdl = pool->tuning.serial_launch == 0 || pool->tuning.serial_launch == 3;
   return launch_projection(a, (cudaStream_t)stream);
 }
 
@@ -178,8 +178,11 @@ static int decode_attend(dkv_pool* pool, int layer, const int32_t* block_table, 
   a.vnew = reinterpret_cast<const float*>(ws + w.off_vnew);
   a.out = out;
   a.lsu_hbm = pool->tuning.attn_lsu_hbm;
-  a.pdl = !pool->tuning.serial_launch;
+  a.pdl = pool->tuning.serial_launch != 1;
   a.early_kv = early_kv && a.pdl;
+  a.signal_next = pool->tuning.serial_launch == 0 || pool->tuning.serial_launch == 3;
+  a.wait_ns = pool->tuning.wait_limit_us > 0 ? (uint64_t)pool->tuning.wait_limit_us * 1000ull : 4000000000ull;
+  a.withhold = pool->tuning.test_withhold_block != 0;
   return launch_attention(a, B, w.Hkv, w.D, w.G, resolve_attn_variant(pool, B, w.Hkv, w.G, max_blocks),
                           (cudaStream_t)stream);
 }

@@ -13,9 +13,12 @@
 //   * naive zero-copy  (DKV_GEMM_NAIVE_ZERO_COPY): row-major tile order. CTAs running at the
 //     same time share an A row panel (L2-resident) but each needs a different B column
 //     panel, so every M tile row re-reads B over the host link.
-//   * CPU-aware        (DKV_GEMM_CPU_AWARE): B-panel-major order. All M tiles of one B
-//     column panel run together, so each B tile crosses the host link once and is served
-//     from L2 to the other tiles; A is re-streamed from HBM once per column panel.
+//   * CPU-aware        (DKV_GEMM_CPU_AWARE): B-panel-major order. Two fetcher warps per
+//     CTA copy each 256-column B panel from host memory into a rotating HBM panel buffer
+//     (kGPanelBufs buffers of [256][K]) exactly once, publishing per-panel readiness; the
+//     M tiles of that panel then read B from the buffer in HBM, so each B element crosses
+//     the host link once (the L2 alone does not keep repeated host reads off the link);
+//     A is re-streamed from HBM once per column panel.
 //   * staged swap      (DKV_GEMM_STAGED_SWAP): cudaMemcpyAsync of the whole B into a
 //     device workspace, then the kernel on device-resident operands.
 //   * device           (DKV_GEMM_DEVICE): both operands already in device memory.

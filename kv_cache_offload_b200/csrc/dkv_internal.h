@@ -67,9 +67,13 @@ struct AttnParams {
   const float* knew; // [B][Hkv][D]
   const float* vnew; // [B][Hkv][D]
   uint16_t* out;     // [B][Hq*D] bf16, or nullptr
-  int lsu_hbm;       // load HBM-tier blocks with cp.async instead of bulk copies
+  int lsu_hbm;       // bit 0: HBM-tier blocks by cp.async instead of bulk copies; bit 1:
+                     // host-tier blocks by bulk copies instead of cp.async
   int pdl;           // launch with programmatic dependent launch
   int early_kv;      // the kernel ahead is this step's projection: stream KV before it ends
+  int signal_next;   // let the next kernel in the stream launch early (programmatic launch)
+  uint64_t wait_ns;  // limit of each bounded wait
+  int withhold;      // test hook: CTA (0, 0, 0) withholds its first block (bounded-wait test)
 };
 
 int launch_attention(const AttnParams& p, int B, int Hkv, int D, int G, int variant, cudaStream_t st);
@@ -102,6 +106,12 @@ int launch_projection(const ProjArgs& a, cudaStream_t st);
 
 // 2-D bf16 tensor map over a row-major [rows][cols] array, box [box_rows][64], 128B swizzle.
 int encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
+// NUMA placement of the host tier (dkv_numa.cu).
+int numa_node_of_pci(const char* sysfs_root, const char* pci_bus_id);
+int gpu_numa_node(int device);
+struct SavedPolicy;
+int alloc_host_on_node(size_t bytes, unsigned flags, int node, void** out);
 
 // Workspace carve-up of one decode step (all offsets 256-byte aligned).
 struct DecodeWs {

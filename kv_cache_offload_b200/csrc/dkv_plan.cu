@@ -47,8 +47,12 @@ __device__ __forceinline__ void apply_plan_body(const PoolView& pool, const uint
       if (threadIdx.x == 0 && layer == 0) flag_error(pool.status, kErrBadBlock);
       continue;
     }
-    const uint4* src = reinterpret_cast<const uint4*>(tier_base(pool, mv.x) + chunk_offset(pool, mv.x, layer, mv.y, 0, 0));
-    uint4* dst = reinterpret_cast<uint4*>(tier_base(pool, mv.z) + chunk_offset(pool, mv.z, layer, mv.w, 0, 0));
+    const int64_t so = chunk_offset(pool, mv.x, layer, mv.y, 0, 0), dof = chunk_offset(pool, mv.z, layer, mv.w, 0, 0);
+    if (!DKV_DEBUG_RANGE(pool.status, so, so + chunk16 * 8, tier_elems(pool, mv.x)) ||
+        !DKV_DEBUG_RANGE(pool.status, dof, dof + chunk16 * 8, tier_elems(pool, mv.z)))
+      continue;
+    const uint4* src = reinterpret_cast<const uint4*>(tier_base(pool, mv.x) + so);
+    uint4* dst = reinterpret_cast<uint4*>(tier_base(pool, mv.z) + dof);
     int64_t c = threadIdx.x;
     for (; c + 3 * 256 < chunk16; c += 4 * 256) {
       const uint4 r0 = __ldcs(src + c), r1 = __ldcs(src + c + 256), r2 = __ldcs(src + c + 512),

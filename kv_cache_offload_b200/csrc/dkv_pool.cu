@@ -59,8 +59,9 @@ __global__ void append_kv_kernel(PoolView pool, int layer, const uint16_t* __res
     if (tier > 1) { flag_error(pool.status, kErrBadTier); continue; }
     if (phys < 0 || phys >= tier_blocks(pool, tier)) { flag_error(pool.status, kErrBadBlock); continue; }
     const uint16_t* src = (kv ? v : k) + (((int64_t)b * n_tokens + t) * pool.Hkv + g) * pool.D + pc * 8;
-    uint16_t* dst = tier_base(pool, tier) + chunk_offset(pool, tier, layer, phys, kv, g) +
-                    (int64_t)slot * pool.D + pc * 8;
+    const int64_t o = chunk_offset(pool, tier, layer, phys, kv, g) + (int64_t)slot * pool.D + pc * 8;
+    if (!DKV_DEBUG_RANGE(pool.status, o, o + 8, tier_elems(pool, tier))) continue;
+    uint16_t* dst = tier_base(pool, tier) + o;
     *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
   }
 }
@@ -117,8 +118,13 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(PoolView pool, int src
         if (c == 0 && l == 0) flag_error(pool.status, kErrBadBlock);
         continue;
       }
-      const uint4* src = reinterpret_cast<const uint4*>(tier_base(pool, src_tier) + chunk_offset(pool, src_tier, l, s, 0, 0)) + c;
-      dst[u] = reinterpret_cast<uint4*>(tier_base(pool, dst_tier) + chunk_offset(pool, dst_tier, l, d, 0, 0)) + c;
+      const int64_t so = chunk_offset(pool, src_tier, l, s, 0, 0) + c * 8;
+      const int64_t dof = chunk_offset(pool, dst_tier, l, d, 0, 0) + c * 8;
+      if (!DKV_DEBUG_RANGE(pool.status, so, so + 8, tier_elems(pool, src_tier)) ||
+          !DKV_DEBUG_RANGE(pool.status, dof, dof + 8, tier_elems(pool, dst_tier)))
+        continue;
+      const uint4* src = reinterpret_cast<const uint4*>(tier_base(pool, src_tier) + so);
+      dst[u] = reinterpret_cast<uint4*>(tier_base(pool, dst_tier) + dof);
       v[u] = __ldcs(src);
     }
 #pragma unroll
@@ -143,7 +149,7 @@ int dkv_pool_create(const dkv_pool_config* cfg, dkv_pool** out) {
   const dkv_pool_config& c = *cfg;
   if (c.num_layers < 1 || c.num_kv_heads < 1 || c.hbm_blocks < 0 || c.host_blocks < 0 ||
       (c.layout != DKV_LAYOUT_LAYER_FIRST && c.layout != DKV_LAYOUT_PAGE_FIRST) ||
-      (c.host_flags & ~DKV_HOST_WRITE_COMBINED))
+      (c.host_flags & ~(DKV_HOST_WRITE_COMBINED | DKV_HOST_NUMA_NEAREST)))
     return set_error(DKV_ERR_ARG, "dkv_pool_create: invalid geometry");
   if ((c.head_dim != 64 && c.head_dim != 128) || c.block_tokens != 16)
     return set_error(DKV_ERR_UNSUPPORTED, "dkv_pool_create: need head_dim 64|128, block_tokens 16");
@@ -190,7 +196,9 @@ int dkv_pool_create(const dkv_pool_config* cfg, dkv_pool** out) {
     unsigned flags = cudaHostAllocMapped | cudaHostAllocPortable;
     if (c.host_flags & DKV_HOST_WRITE_COMBINED) flags |= cudaHostAllocWriteCombined;
     void* h = nullptr;
-    e = cudaHostAlloc(&h, p->host_bytes, flags);
+    const int node = (c.host_flags & DKV_HOST_NUMA_NEAREST) ? gpu_numa_node(dev) : -1;
+    const int arc = alloc_host_on_node(p->host_bytes, flags, node, &h);
+    e = arc == DKV_OK ? cudaSuccess : (cudaError_t)arc;
     if (e != cudaSuccess) {
       cudaGetLastError();
       if (p->own_hbm) cudaFree(p->hbm);
@@ -251,8 +259,9 @@ int dkv_pool_set_tuning(dkv_pool* p, const dkv_tuning* t) {
   if (!p) return set_error(DKV_ERR_ARG, "dkv_pool_set_tuning: null pool");
   if (t) {
     const int v = t->attn_variant;
-    if (t->attn_splits < 0 || t->proj_splits < 0 || t->proj_splits > 16 || (v != 0 && v != 1 && v != 2 && v != 5 && v != 6 && v != 7) ||
-        t->attn_lsu_hbm < 0 || t->attn_lsu_hbm > 1 || t->serial_launch < 0 || t->serial_launch > 1)
+    if (t->attn_splits < 0 || t->proj_splits < 0 || t->proj_splits > 16 || (v != 0 && v != 1 && v != 5 && v != 6 && v != 7 && v != 8 && v != 9) ||
+        t->attn_lsu_hbm < 0 || t->attn_lsu_hbm > 3 || t->serial_launch < 0 || t->serial_launch > 3 ||
+        t->wait_limit_us < 0 || t->test_withhold_block < 0 || t->test_withhold_block > 1)
       return set_error(DKV_ERR_ARG, "dkv_pool_set_tuning: value out of range");
     p->tuning = *t;
   } else {
@@ -394,6 +403,8 @@ int dkv_check(dkv_pool* p, void* stream) {
   if (rc) return rc;
   if (!word) return DKV_OK;
   cudaMemset(p->d_status, 0, sizeof(int));
+  if (word & kErrDebugBounds)
+    return set_error(DKV_ERR_INTERNAL, "a debug-build range check failed in a kernel (status 0x%x)", word);
   if (word & kErrTimeout)
     return set_error(DKV_ERR_TIMEOUT, "device wait timed out (status 0x%x)", word);
   return set_error(DKV_ERR_BAD_TABLE, "device rejected table entries (status 0x%x:%s%s%s%s)", word,

@@ -13,13 +13,17 @@
 //    CTA streams its slice of the tile once through a TMA ring (128-byte swizzle, one
 //    elected thread issues tcgen05.mma M=128, N, K=16 per 16 columns). Clusters are small
 //    and CTAs light (two per SM), so the whole GPU streams W concurrently.
-//  * Each CTA moves its partial [128 x N] accumulator TMEM -> shared memory; after a
-//    cluster barrier, CTA r sums batch columns b = r, r + CS, ... over the CS partials in
-//    rank order through distributed shared memory (a fixed order: deterministic), then
-//    finishes those columns: q heads rotated and scaled by log2(e)/sqrt(D) for the
-//    log2-domain softmax, the key head rotated and rounded to bf16 (k_hat), the value
-//    head rounded (v_hat); k_hat and v_hat are written once into the cache slot and, as
-//    fp32, into the workspace for the new token's attention term.
+//  * While W streams, the otherwise idle warps look up, for every batch column b the CTA
+//    will finish (b = r, r + CS, ... for cluster rank r), its position and cache-slot
+//    addresses, and compute the RoPE (cos, sin) of each rotation pair at that position.
+//  * Each CTA then reads its partial [128 x N] accumulator from TMEM and stores column b
+//    straight into the shared memory of the CTA that finishes it (distributed shared
+//    memory, rank b mod CS); after one cluster barrier every CTA sums its columns over the
+//    CS partials in rank order from its own shared memory (a fixed order: deterministic)
+//    and finishes them: q heads rotated and scaled by log2(e)/sqrt(D) for the log2-domain
+//    softmax, the key head rotated and rounded to bf16 (k_hat), the value head rounded
+//    (v_hat); k_hat and v_hat are written once into the cache slot and, as fp32, into the
+//    workspace for the new token's attention term.
 // Reading W is the whole cost (HBM-bound); the tensor cores only remove the CUDA-core FMA
 // bound that B >= 16 would otherwise hit.
 #include <cooperative_groups.h>
@@ -46,6 +50,8 @@ struct ProjParams {
   int max_blocks;
   int B, H, Hq, Hkv, D, G;
   int ppt, nt, Npad, CS, KB, nst;
+  int slots;                           // batch columns a CTA finishes: ceil(B / CS)
+  int off_recv, off_rope, off_cols, off_bars;  // shared-memory carve-up (bytes)
   float qscale;
   float* qs;              // [B][Hq][D]
   float* knew;            // [B][Hkv][D]
@@ -55,23 +61,23 @@ struct ProjParams {
 };
 
 // Distributed-shared-memory access: address of `p` in CTA `rank` of the cluster, and a
-// 32-bit load through that address.
+// 32-bit store through that address.
 __device__ __forceinline__ uint32_t dsmem_map(const void* p, int rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float dsmem_ld(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
+__device__ __forceinline__ void dsmem_st(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
-// Epilogue lookups done while W streams, for the first four sequences a CTA finishes:
-// the position and the two cache-slot addresses (key, value) of kv head g.
-struct EpiPre {
-  int pos[4];
-  uint16_t* dst[4][2];
+// Epilogue lookups done while W streams, one per batch column the CTA finishes: the
+// position and the two cache-slot addresses (key, value) of kv head g (null where the
+// table entry was rejected and flagged).
+struct EpiCol {
+  uint16_t* dst[2];
+  int pos;
+  int pad;
 };
 
 // First W row of piece (head) `pc` of kv-head group g: pieces 0..G-1 are the group's q
@@ -92,18 +98,21 @@ __global__ void __launch_bounds__(kPThreads, 2)
   const int g = tile / p.nt, t = tile % p.nt;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // 1024-byte aligned carve-up: ring | barriers | tmem slot | epilogue lookups
+  // 1024-byte aligned carve-up: ring | column receive area | RoPE table | column lookups |
+  // barriers | tmem slot
   const uint32_t base_u = smem_u32(psmem_raw);
   uint8_t* smem = psmem_raw + (((base_u + 1023u) & ~1023u) - base_u);
   const int xtile = p.Npad * 128;
   const int stage_bytes = kWTile + xtile;
   const int nst = p.nst;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + nst * stage_bytes);
+  const int slots = p.slots;
+  float* recv = reinterpret_cast<float*>(smem + p.off_recv);     // [CS][slots][128] partial columns
+  float2* rope = reinterpret_cast<float2*>(smem + p.off_rope);   // [slots][D/2] (cos, sin)
+  EpiCol* cols = reinterpret_cast<EpiCol*>(smem + p.off_cols);   // [slots]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bars);
   uint64_t* empty = full + nst;
   uint64_t* done = empty + nst;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
-  float* part = reinterpret_cast<float*>(smem);  // [Npad][128], aliases the ring later
-  EpiPre* pre = reinterpret_cast<EpiPre*>(smem + nst * stage_bytes + 128);  // after the barriers
 
   if (tid == 0) {
     for (int i = 0; i < nst; ++i) {
@@ -165,18 +174,21 @@ __global__ void __launch_bounds__(kPThreads, 2)
       umma_commit(&empty[st]);
     }
     umma_commit(done);
-  } else {
-    // the tables, positions and workspace below belong to the kernels ahead in the stream
+  } else if (warp >= 2) {
+    // ------------------------------------ epilogue tables, while W streams (warps 2, 3)
+    // the tables and positions belong to the kernels ahead in the stream
     griddep_wait();
     if (tid == 64) griddep_launch_dependents();
-    if (tid >= 64 && tid < 68) {
-      // while W streams: position and cache-slot addresses of sequence rank + CS * i
-      const int i = tid - 64, b = rank + p.CS * i;
-      int pos = 0;
-      uint16_t* dk = nullptr;
-      uint16_t* dv = nullptr;
+    const int et = tid - 64;
+    for (int it = et; it < slots; it += 64) {  // position and cache-slot addresses per column
+      const int b = rank + p.CS * it;
+      EpiCol c;
+      c.dst[0] = c.dst[1] = nullptr;
+      c.pos = 0;
+      c.pad = 0;
       if (b < p.B) {
-        pos = p.seq_lens[b];
+        const int pos = p.seq_lens[b];
+        c.pos = pos;
         const int64_t jb = pos >= 0 ? (int64_t)pos / p.pool.T : -1;
         if (jb < 0 || jb >= p.max_blocks) {
           flag_error(p.pool.status, kErrCtxTooLong);
@@ -189,33 +201,59 @@ __global__ void __launch_bounds__(kPThreads, 2)
             flag_error(p.pool.status, kErrBadBlock);
           } else {
             const int64_t slot = (int64_t)(pos % p.pool.T) * p.D;
-            dk = tier_base(p.pool, tier) + chunk_offset(p.pool, tier, p.layer, phys, 0, g) + slot;
-            dv = tier_base(p.pool, tier) + chunk_offset(p.pool, tier, p.layer, phys, 1, g) + slot;
+            const int64_t ok = chunk_offset(p.pool, tier, p.layer, phys, 0, g) + slot;
+            const int64_t ov = chunk_offset(p.pool, tier, p.layer, phys, 1, g) + slot;
+            const int64_t n = tier_elems(p.pool, tier);
+            if (DKV_DEBUG_RANGE(p.pool.status, ok, ok + p.D, n) && DKV_DEBUG_RANGE(p.pool.status, ov, ov + p.D, n)) {
+              c.dst[0] = tier_base(p.pool, tier) + ok;
+              c.dst[1] = tier_base(p.pool, tier) + ov;
+            }
           }
         }
       }
-      pre->pos[i] = pos;
-      pre->dst[i][0] = dk;
-      pre->dst[i][1] = dv;
+      cols[it] = c;
+    }
+    if (t * p.ppt <= p.G) {  // the tile holds q or key heads: RoPE (cos, sin) per column and pair
+      // rotate-half RoPE: angle pos * theta^(-2i/D) reduced mod 2*pi in fp64, then a
+      // single-precision sincos
+      const int half = p.D / 2;
+      for (int e = et; e < slots * half; e += 64) {
+        const int it = e / half, pi = e % half;
+        const int b = rank + p.CS * it;
+        if (b >= p.B) continue;
+        const double ang = (double)p.seq_lens[b] * p.inv_freq[pi];
+        const double red = ang - rint(ang * 0.15915494309189535) * 6.283185307179586;
+        float sn, cn;
+        sincosf((float)red, &sn, &cn);
+        rope[e] = make_float2(cn, sn);
+      }
     }
   }
   __syncwarp();
   griddep_wait();
 
-  // ----------------------------------------------------- TMEM -> shared partial [n][row]
+  // -------------------------------- TMEM -> the shared memory of each column's finisher
+  // column b goes to cluster rank b mod CS, slot b / CS, as its row-`tid` element
   mbar_wait_bounded(done, 0, p.pool.status);
   tc_fence_after();
   for (int c0 = 0; c0 < p.Npad; c0 += 16) {
     float v[16];
     tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) part[(c0 + j) * 128 + tid] = v[j];
+    for (int j = 0; j < 16; ++j) {
+      const int b = c0 + j;
+      if (b < p.B)
+        dsmem_st(dsmem_map(recv + ((size_t)(rank * slots + b / p.CS) * 128 + tid), b % p.CS), v[j]);
+    }
   }
   tc_fence_before();
   if (t == 0 && rank == 0 && tid < p.B && p.attn_cnt) p.attn_cnt[(int64_t)tid * p.Hkv + g] = 0;
-  cluster.sync();  // every CTA's partial is in its shared memory
+  cluster.sync();  // every partial column has arrived where it is finished (and no CTA
+                   // touches another's shared memory after this)
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 32);
 
-  // ------------------------------------ column reduction over the cluster + epilogue
+  // ------------------------------------ column reduction (rank order) + epilogue
   // thread -> tile row (head row / D of the tile, dim d = row % D of that head), mapped so
   // that the two rows of a RoPE pair (d and d + D/2) sit in lanes l and l ^ 16 of one
   // warp: the pair exchange is a shuffle, with no block barrier per sequence
@@ -224,27 +262,16 @@ __global__ void __launch_bounds__(kPThreads, 2)
   const int pc = t * p.ppt + row / D;     // piece (head) index within the group
   const int d = row % D, pi = d % half;   // RoPE pair index
   const bool live = row / D < np;
-  uint32_t rbase[16];
-#pragma unroll
-  for (int q = 0; q < 16; ++q) rbase[q] = dsmem_map(part, q < p.CS ? q : 0);
-  for (int b = rank, it = 0; b < p.B; b += p.CS, ++it) {
-    const uint32_t off = (uint32_t)((b * 128 + row) * 4);
-    float vals[16];
-#pragma unroll
-    for (int q = 0; q < 16; ++q) vals[q] = q < p.CS ? dsmem_ld(rbase[q] + off) : 0.f;
+  for (int it = 0; it < slots; ++it) {
+    const int b = rank + p.CS * it;
+    if (b >= p.B) break;
     float x = 0.f;
-#pragma unroll
-    for (int q = 0; q < 16; ++q) x += vals[q];  // rank order: deterministic
+    for (int q = 0; q < p.CS; ++q) x += recv[(q * slots + it) * 128 + row];  // rank order: deterministic
     const float xp = __shfl_xor_sync(0xffffffffu, x, 16);  // the pair's other row
     if (!live) continue;
-    const int pos = it < 4 ? pre->pos[it] : p.seq_lens[b];
     if (pc <= p.G) {
-      // rotate-half RoPE: angle reduced mod 2*pi in fp64, then a single-precision sincos
-      const double ang = (double)pos * p.inv_freq[pi];
-      const double red = ang - rint(ang * 0.15915494309189535) * 6.283185307179586;
-      float sn, cn;
-      sincosf((float)red, &sn, &cn);
-      const float y = d < half ? x * cn - xp * sn : x * cn + xp * sn;
+      const float2 cs = rope[it * half + pi];
+      const float y = d < half ? x * cs.x - xp * cs.y : x * cs.x + xp * cs.y;
       if (pc < p.G) {
         p.qs[((int64_t)b * p.Hq + g * p.G + pc) * D + d] = y * p.qscale;
         continue;
@@ -254,31 +281,11 @@ __global__ void __launch_bounds__(kPThreads, 2)
     const uint16_t hb = f32_to_bf16_bits(x);
     const int kv = pc == p.G ? 0 : 1;
     (kv ? p.vnew : p.knew)[((int64_t)b * p.Hkv + g) * D + d] = __uint_as_float((uint32_t)hb << 16);
-    // the single cache write: slot pos mod T of logical block pos / T (looked up while W
-    // streamed for the first four sequences; bad entries were flagged there)
-    if (it < 4) {
-      if (pre->dst[it][kv]) pre->dst[it][kv][d] = hb;
-      continue;
-    }
-    const int64_t jb = pos >= 0 ? (int64_t)pos / p.pool.T : -1;
-    if (jb < 0 || jb >= p.max_blocks) {
-      flag_error(p.pool.status, kErrCtxTooLong);
-      continue;
-    }
-    const int tier = p.tier_map[(int64_t)b * p.max_blocks + jb];
-    const int64_t phys = p.table[(int64_t)b * p.max_blocks + jb];
-    if (tier > 1) {
-      flag_error(p.pool.status, kErrBadTier);
-      continue;
-    }
-    if (phys < 0 || phys >= tier_blocks(p.pool, tier)) {
-      flag_error(p.pool.status, kErrBadBlock);
-      continue;
-    }
-    tier_base(p.pool, tier)[chunk_offset(p.pool, tier, p.layer, phys, kv, g) + (int64_t)(pos % p.pool.T) * D + d] = hb;
+    // the single cache write: slot pos mod T of logical block pos / T (bad entries were
+    // flagged by the lookup and are skipped)
+    uint16_t* dst = cols[it].dst[kv];
+    if (dst) dst[d] = hb;
   }
-  cluster.sync();  // no CTA leaves while others may still read its partial
-  if (warp == 0) tmem_dealloc(tmem, 32);
 }
 
 // ------------------------------------------------------------------ host side
@@ -310,8 +317,24 @@ int encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t col
   return DKV_OK;
 }
 
-static size_t proj_smem_bytes(int Npad, int nst) {
-  return 1024 + (size_t)nst * (kWTile + Npad * 128) + 256;
+// Shared memory per CTA: two CTAs share an SM (228 KB, 1 KB of it reserved per CTA).
+constexpr int kProjSmemBudget = 113 * 1024;
+
+// Carve-up of one CTA's shared memory for a ring of `nst` stages; returns the total
+// (including the 1024-byte alignment slack).
+static int proj_smem_layout(ProjParams* p, int nst) {
+  const int stage = kWTile + p->Npad * 128;
+  int o = nst * stage;
+  p->off_recv = o;
+  o += p->CS * p->slots * 128 * 4;
+  p->off_rope = o;
+  o += p->slots * (p->D / 2) * 8;
+  p->off_cols = o;
+  o += p->slots * (int)sizeof(EpiCol);
+  o = (o + 7) / 8 * 8;
+  p->off_bars = o;
+  o += (2 * nst + 1) * 8 + 8;
+  return 1024 + o;
 }
 
 int launch_projection(const ProjArgs& a, cudaStream_t st) {
@@ -327,7 +350,6 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
   p.ppt = 128 / a.D;
   p.nt = (p.G + 2 + p.ppt - 1) / p.ppt;
   p.Npad = a.B <= 16 ? 16 : 32;
-  p.nst = p.Npad == 16 ? 6 : 5;  // ring fits two CTAs per SM
   p.KB = a.H / 64;
   for (int i = 0; i < a.D / 2; ++i) p.inv_freq[i] = pow(a.theta, -2.0 * (double)i / (double)a.D);
   p.attn_cnt = a.attn_cnt;
@@ -335,8 +357,6 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
   p.qs = a.qs;
   p.knew = a.knew;
   p.vnew = a.vnew;
-  const size_t smem = proj_smem_bytes(p.Npad, p.nst);
-
   CUtensorMap tmW, tmX;
   int rc = encode_bf16_2d(&tmW, a.W, (uint64_t)(a.Hq + 2 * a.Hkv) * a.D, a.H, (uint32_t)a.D);
   if (rc) return rc;
@@ -345,9 +365,8 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
 
   static bool attr = false;
   if (!attr) {
-    const size_t mx = proj_smem_bytes(16, 6) > proj_smem_bytes(32, 5) ? proj_smem_bytes(16, 6)
-                                                                      : proj_smem_bytes(32, 5);
-    cudaError_t e = cudaFuncSetAttribute(proj_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mx);
+    cudaError_t e = cudaFuncSetAttribute(proj_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kProjSmemBudget);
     if (e != cudaSuccess) return cuda_check(e, "projection: smem attribute");
     attr = true;
   }
@@ -358,6 +377,14 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
   if (CS < 1) CS = 1;
   if (CS > 8) CS = 8;
   if (CS > p.KB) CS = p.KB;
+  p.CS = CS;
+  p.slots = (a.B + CS - 1) / CS;
+  // the deepest ring (3..6 stages) that leaves room for the epilogue areas at two CTAs/SM
+  int nst = 6;
+  while (nst > 3 && proj_smem_layout(&p, nst) > kProjSmemBudget) --nst;
+  const int smem = proj_smem_layout(&p, nst);
+  if (smem > kProjSmemBudget) return set_error(DKV_ERR_UNSUPPORTED, "projection: shared memory (%d B)", smem);
+  p.nst = nst;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[2] = {};
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -372,7 +399,6 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = a.pdl ? 2 : 1;
-  p.CS = CS;
   cudaError_t e = cudaLaunchKernelEx(&cfg, proj_umma_kernel, tmW, tmX, p);
   return cuda_check(e, "projection launch");
 }

@@ -21,6 +21,15 @@ def test_every_declared_symbol_is_exported():
     assert not missing, missing
 
 
+def test_debug_library_exports_the_same_symbols():
+    # libdkv_debug.so: the same sources with DKV_DEBUG range checks (loaded with
+    # DKV_LIBRARY=debug); it must offer every call the header declares
+    from kv_cache_offload_b200.build import LIB_DEBUG
+    L = ctypes.CDLL(LIB_DEBUG)
+    missing = [n for n in dkv.header_symbols() if not hasattr(L, n)]
+    assert not missing, missing
+
+
 def test_binding_declares_every_symbol():
     from kv_cache_offload_b200 import binding
     assert set(dkv.header_symbols()) <= set(binding._SIGS)

@@ -47,3 +47,18 @@ def test_workload_config_names_the_workload_without_model_keys():
     assert c["global_batch"] == 32 and c["seq_len"] == 32768 and c["parallelism"] == "replicas x2"
     assert c["workload"].startswith("8b_hbm: B=16 hidden=4096 Hq=32 Hkv=8 D=128")
     assert "model" not in c
+
+
+def test_percentiles_nearest_rank():
+    assert bench.percentiles([5.0, 1.0, 3.0, 2.0, 4.0, 6.0, 7.0, 8.0, 9.0, 10.0]) == [1.0, 5.0, 9.0]
+    assert bench.percentiles([2.0]) == [2.0, 2.0, 2.0]
+
+
+def test_oracle_pool_runs_one_sequence_per_process():
+    # the CPU baseline's process pool on the tiny workload: 2 single-threaded processes;
+    # steps mode returns one wall time per step, budget mode a summed rate
+    cfg = WL.CONFIGS["tiny"]
+    times = bench.run_oracle_pool(cfg, 0, 2, steps=3)
+    assert len(times) == 3 and all(t > 0 for t in times)
+    rate, done, el = bench.run_oracle_pool(cfg, 0, 2, budget_s=0.2)
+    assert done >= 2 and rate > 0 and el >= 0.2

@@ -125,6 +125,32 @@ def test_bad_table_entries_are_flagged_not_fatal():
         ctx.close()
 
 
+@pytest.mark.parametrize("variant", [5, 1, 6])
+def test_bounded_wait_gives_up_and_the_pool_stays_usable(variant):
+    # a stage that is never loaded (the test hook withholds the first block of CTA (0, 0, 0)):
+    # its consumer's bounded wait gives up after 2 ms, the kernel returns, dkv_check reports
+    # DKV_ERR_TIMEOUT; the other sequence's output is unaffected and the next step is exact
+    cfg = WL.small_config(B=2, Hq=8, Hkv=2, ctx_range=(600, 800), host_prob=0.3, layers=1)
+    inp = WL.make_decode_inputs(cfg, seed=12)
+    ctx = TL.make_pool(inp)
+    try:
+        x, W = inp.x.cuda(), inp.W.cuda()
+        out = torch.empty((cfg.B, cfg.Hq * cfg.D), dtype=torch.bfloat16, device="cuda")
+        dkv.dkv_pool_set_tuning(ctx.pool, attn_splits=1, attn_variant=variant, wait_limit_us=2000,
+                                test_withhold_block=1)
+        nws = dkv.dkv_decode_workspace_bytes(ctx.pool, cfg.B, ctx.table.shape[1], cfg.Hq, cfg.H)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        dkv.dkv_decode_step(ctx.pool, 0, x, W, ctx.table, ctx.seq_lens, ctx.tier_map, cfg.Hq, cfg.theta, out, ws)
+        assert dkv.dkv_check(ctx.pool) == dkv.DKV_ERR_TIMEOUT
+        assert "timed out" in dkv.dkv_last_error()
+        TL.assert_out_close(out, TL.oracle_step(inp, batch=[1])["out"], "sequence 1 beside a timed-out CTA")
+        assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK  # the status word was cleared
+        good = TL.run_step(ctx)  # default tuning again (run_step asserts DKV_OK)
+        TL.assert_out_close(good, TL.oracle_step(inp)["out"], "step after the timeout")
+    finally:
+        ctx.close()
+
+
 def test_argument_errors():
     cfg = WL.small_config(B=2)
     inp = WL.make_decode_inputs(cfg)
@@ -219,7 +245,7 @@ def test_staged_calls_match_fused_step():
         ctx.close()
 
 
-@pytest.mark.parametrize("variant", [1, 2, 5, 6, 7])  # 0 (automatic) is 1
+@pytest.mark.parametrize("variant", [1, 5, 6, 7])
 @pytest.mark.parametrize("splits", [1, 0])  # one split: long CTAs that wrap the stage ring
 @pytest.mark.parametrize("D", [64, 128])
 def test_attention_kernel_variants(variant, splits, D):
@@ -238,6 +264,30 @@ def test_attention_kernel_variants(variant, splits, D):
         assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
         TL.assert_out_close(out, TL.oracle_step(inp, layer=1)["out"], "variant %d" % variant)
         # same splits, same reduction order per (slot, head): the variants agree closely
+        assert (out.float() - base.float()).abs().max().item() <= 2 ** -6
+    finally:
+        ctx.close()
+
+
+@pytest.mark.parametrize("variant", [1, 5, 8, 9, 6])
+@pytest.mark.parametrize("splits", [1, 0])
+@pytest.mark.parametrize("D", [64, 128])
+def test_attention_kernel_variants_group_of_8(variant, splits, D):
+    # G = 8 (the 70B shape): two consumer warps of four heads per block in the CUDA-core
+    # shapes; every shape against the oracle, and against each other
+    cfg = WL.small_config(B=3, Hq=16, Hkv=2, D=D, H=256, ctx_range=(300, 700), host_prob=0.5)
+    inp = WL.make_decode_inputs(cfg, seed=13)
+    ctx = TL.make_pool(inp)
+    try:
+        base = TL.run_step(ctx, layer=1)
+        dkv.dkv_pool_set_tuning(ctx.pool, attn_splits=splits, attn_variant=variant)
+        x, W = inp.x.cuda(), inp.W.cuda()
+        out = torch.empty_like(base)
+        nws = dkv.dkv_decode_workspace_bytes(ctx.pool, cfg.B, ctx.table.shape[1], cfg.Hq, cfg.H)
+        ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
+        dkv.dkv_decode_step(ctx.pool, 1, x, W, ctx.table, ctx.seq_lens, ctx.tier_map, cfg.Hq, cfg.theta, out, ws)
+        assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
+        TL.assert_out_close(out, TL.oracle_step(inp, layer=1)["out"], "G=8 variant %d" % variant)
         assert (out.float() - base.float()).abs().max().item() <= 2 ** -6
     finally:
         ctx.close()
@@ -273,23 +323,25 @@ def test_unwritten_tail_slots_are_ignored(D, Hq):
 
 def test_serial_launch_matches_overlapped_launch():
     """Programmatic dependent launch only moves kernel starts: outputs are bit-identical
-    with the kernels launched one after another."""
+    with the kernels launched one after another, and with the overlap kept inside a step."""
     cfg = WL.small_config(B=5, Hq=16, Hkv=2, D=128, H=512, ctx_range=(100, 900), host_prob=0.3)
     inp = WL.make_decode_inputs(cfg, seed=31)
     ctx = TL.make_pool(inp)
     try:
         a = TL.run_step(ctx, layer=1)
-        dkv.dkv_pool_set_tuning(ctx.pool, serial_launch=1)
         x, W = inp.x.cuda(), inp.W.cuda()
-        b = torch.empty_like(a)
         nws = dkv.dkv_decode_workspace_bytes(ctx.pool, cfg.B, ctx.table.shape[1], cfg.Hq, cfg.H)
         ws = torch.empty(nws, dtype=torch.uint8, device="cuda")
-        for _ in range(3):  # back to back on one stream, as a serving loop runs them
-            dkv.dkv_decode_step(ctx.pool, 1, x, W, ctx.table, ctx.seq_lens, ctx.tier_map, cfg.Hq, cfg.theta, b, ws)
-        assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
-        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+        for mode in (1, 2, 3, 0):
+            dkv.dkv_pool_set_tuning(ctx.pool, serial_launch=mode)
+            b = torch.empty_like(a)
+            for _ in range(3):  # back to back on one stream, as a serving loop runs them
+                dkv.dkv_decode_step(ctx.pool, 1, x, W, ctx.table, ctx.seq_lens, ctx.tier_map, cfg.Hq, cfg.theta,
+                                    b, ws)
+            assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16)), mode
         with pytest.raises(dkv.DkvError):
-            dkv.dkv_pool_set_tuning(ctx.pool, serial_launch=2)
+            dkv.dkv_pool_set_tuning(ctx.pool, serial_launch=4)
     finally:
         ctx.close()
 

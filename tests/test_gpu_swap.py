@@ -6,6 +6,7 @@ import pytest
 import torch
 
 import workloads as WL
+from oracle import dkv_oracle as O
 
 pytestmark = pytest.mark.gpu
 
@@ -97,5 +98,13 @@ def test_staged_swap_decode_equals_zero_copy(method):
                             cfg.theta, out, ws)
         assert dkv.dkv_check(pool) == dkv.DKV_OK
         assert torch.equal(out, zc)
+        # against the fp64 oracle: on the original two-tier inputs, and walking the staged
+        # tables over the oracle's own copy of the staged HBM tier (host blocks appended)
+        TL.assert_out_close(out, TL.oracle_step(inp)["out"], "staged vs oracle")
+        staged = np.concatenate([WL.bf16_bits(inp.hbm), WL.bf16_bits(inp.host)], axis=1)
+        ref = O.decode_step(WL.bf16_bits(inp.x), WL.bf16_bits(inp.W), [staged, WL.bf16_bits(inp.host)],
+                            table.numpy(), lay.seq_lens, tmap.numpy(), cfg.Hq, cfg.Hkv, cfg.D, cfg.T,
+                            cfg.theta)["out"]
+        TL.assert_out_close(out, ref, "staged vs oracle on the staged tables")
     finally:
         dkv.dkv_pool_destroy(pool)

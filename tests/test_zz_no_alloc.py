@@ -26,13 +26,6 @@ def _built():
     build()
 
 
-def _close(a: torch.Tensor, b: torch.Tensor):
-    # same bars as the oracle comparisons: max-abs 3e-2, mean-abs 3e-3, rel-rms 1e-2
-    d = (a.float() - b.float()).abs()
-    rel = (a.float() - b.float()).norm() / b.float().norm().clamp_min(1e-30)
-    assert d.max().item() <= 3e-2 and d.mean().item() <= 3e-3 and rel.item() <= 1e-2
-
-
 def test_static_workspace_step_matches_workspace_step_twice():
     cfg = WL.small_config(B=5, ctx_range=(1, 300), host_prob=0.5, layers=2)
     inp = WL.make_decode_inputs(cfg, seed=3)
@@ -40,12 +33,21 @@ def test_static_workspace_step_matches_workspace_step_twice():
     try:
         x, W = inp.x.cuda(), inp.W.cuda()
         ref = TL.run_step(ctx, layer=1)
-        for _ in range(2):  # two calls in a row share (and reuse) the static array
-            out = torch.full_like(ref, float("nan"))
+        outs = [torch.full_like(ref, float("nan")) for _ in range(2)]
+        for i, out in enumerate(outs):  # two calls in a row share (and reuse) the static array
+            torch.cuda.synchronize()
+            free0 = torch.cuda.mem_get_info()[0]
             dkv.dkv_decode_step_static(ctx.pool, 1, x, W, ctx.table, ctx.seq_lens, ctx.tier_map,
                                        cfg.Hq, cfg.theta, out)
+            torch.cuda.synchronize()
+            free1 = torch.cuda.mem_get_info()[0]
             assert dkv.dkv_check(ctx.pool) == dkv.DKV_OK
-            _close(out, ref)
+            # same kernels, split count and workspace layout as the caller-workspace step:
+            # the same bits
+            assert torch.equal(out, ref)
+            if i == 1:  # the first call may commit the array (lazy module loading); later ones nothing
+                assert free1 == free0, "device memory changed across a static-workspace call"
+        TL.assert_out_close(outs[1], TL.oracle_step(inp, layer=1)["out"], "static workspace vs oracle")
     finally:
         ctx.close()
 
@@ -69,5 +71,27 @@ def test_static_workspace_rejects_oversized_shapes():
             dkv.dkv_decode_step_static(ctx.pool, 0, inp.x.cuda(), inp.W.cuda(), table, ctx.seq_lens, tmap,
                                        cfg.Hq, cfg.theta, out)
         assert e.value.code == dkv.DKV_ERR_CAPACITY
+    finally:
+        ctx.close()
+
+
+def test_static_workspace_unsupported_shape_has_the_same_code():
+    # a batch of 33 is beyond the step's limit: both entry points say DKV_ERR_UNSUPPORTED
+    cfg = WL.small_config(B=2, ctx_range=(10, 20), layers=1)
+    inp = WL.make_decode_inputs(cfg)
+    ctx = TL.make_pool(inp)
+    try:
+        B = 33
+        x = torch.zeros((B, cfg.H), dtype=torch.bfloat16, device="cuda")
+        table = torch.zeros((B, 4), dtype=torch.int32, device="cuda")
+        tmap = torch.zeros((B, 4), dtype=torch.uint8, device="cuda")
+        lens = torch.zeros((B,), dtype=torch.int32, device="cuda")
+        out = torch.empty((B, cfg.Hq * cfg.D), dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+        with pytest.raises(dkv.DkvError) as e1:
+            dkv.dkv_decode_step(ctx.pool, 0, x, inp.W.cuda(), table, lens, tmap, cfg.Hq, cfg.theta, out, ws)
+        with pytest.raises(dkv.DkvError) as e2:
+            dkv.dkv_decode_step_static(ctx.pool, 0, x, inp.W.cuda(), table, lens, tmap, cfg.Hq, cfg.theta, out)
+        assert e1.value.code == e2.value.code == dkv.DKV_ERR_UNSUPPORTED
     finally:
         ctx.close()

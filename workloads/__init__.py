@@ -15,6 +15,8 @@ concrete configurations:
             the tail block in HBM, older blocks in the host tier, physical ids permuted
   70b_mixed B=32, H=8192, Hq=64, Hkv=8, D=128, theta=5e5, ctx ~ U{8192..65536}, each
             logical block host-resident with probability 0.8, physical ids permuted
+  70b_hbm   the 70b_mixed layer and lengths with every block in HBM (an added case for
+            the group-size-8 attention against the HBM roofline)
   gemm      M=N=K=10240 bf16, A in HBM, B in the host tier, entries ~ U(-1, 1)
 
 Seeding: one CPU ``torch.Generator`` per tensor, seeded ``seed + index`` with the index
@@ -73,6 +75,10 @@ CONFIGS = {
     "70b_mixed": DecodeConfig("70b_mixed", B=32, H=8192, Hq=64, Hkv=8, D=128, theta=5e5,
                               ctx=None, ctx_range=(8192, 65536), tier_policy="bernoulli",
                               host_prob=0.8, permute=True),
+    # the same 70B-shaped layer with every block in HBM: the group size 8 attention
+    # against the HBM roofline (an added measurement case, not one of the five above)
+    "70b_hbm": DecodeConfig("70b_hbm", B=32, H=8192, Hq=64, Hkv=8, D=128, theta=5e5,
+                            ctx=None, ctx_range=(8192, 65536), tier_policy="hbm", permute=True),
 }
 
 
