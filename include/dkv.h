@@ -85,16 +85,14 @@ typedef struct dkv_tuning {
   int32_t attn_splits;   /* split-K factor of the attention grid (per sequence, kv head) */
   int32_t proj_splits;   /* cluster size of the projection (its reduction split), <= 16 */
   int32_t attn_variant;  /* attention kernel: 0 automatic (see dkv_decode_attn_variant),
-                            5 CUDA-core products with q in registers, three consumer slots
-                            and a 6-stage ring (G <= 4: one warp per slot, 4 CTAs/SM;
-                            G = 8: two warps per slot, 2 CTAs/SM), 1 CUDA cores with four
-                            slots and an 8-stage ring (3 CTAs/SM; G = 8: two warps per
-                            slot, 1 CTA/SM), 8 (G = 8 only, else as 1) two slots of two
-                            warps, a 4-stage ring, 3 CTAs/SM, 6 tensor-core products
-                            (4-stage ring, 4 CTAs/SM), 7 tensor cores with an 8-stage
-                            ring (3 CTAs/SM); other values are invalid. The tensor-core
-                            consumers are opt-in: the design reserves the tensor cores
-                            for the projection */
+                            5 CUDA-core products with q in registers (G <= 4: three
+                            one-warp consumer slots, a 6-stage ring, 4 CTAs/SM; G = 8: two
+                            slots of two warps, a 4-stage ring, 3 CTAs/SM), 1 CUDA cores
+                            with four slots and an 8-stage ring (3 CTAs/SM; G = 8: slots of
+                            two warps, 1 CTA/SM), 6 tensor-core products (4-stage ring,
+                            4 CTAs/SM), 7 tensor cores with an 8-stage ring (3 CTAs/SM);
+                            other values are invalid. The tensor-core consumers are opt-in:
+                            the design reserves the tensor cores for the projection */
   int32_t attn_lsu_hbm;  /* load paths of the CUDA-core attention, bits: 1 = HBM-tier blocks
                             by 16-byte cp.async instead of bulk copies (TMA engine); 2 =
                             host-tier blocks by bulk copies from the mapped host memory
@@ -287,8 +285,8 @@ size_t dkv_decode_static_workspace_capacity(void);
 int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 
 /* The attention kernel variant dkv_decode_step runs for this shape: the pool's
- * dkv_tuning.attn_variant, or, when that is 0, the automatic choice (for Hq/Hkv = 4: 5 when
- * its split-K ranges keep at least 100 blocks of the table each, else 1; 1 otherwise).
+ * dkv_tuning.attn_variant, or, when that is 0, the automatic choice (for Hq/Hkv = 4 or 8: 5
+ * when its split-K ranges keep at least 100 blocks of the table each, else 1; 1 otherwise).
  * Returns the variant (> 0) or a negative DKV_ERR_* code. */
 int dkv_decode_attn_variant(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 

@@ -369,13 +369,10 @@ __device__ __forceinline__ int longest_first_sequence(const AttnParams& p, int* 
   return *s_b;
 }
 
-// QSM: q in shared memory instead of registers (the group-of-8 shape with one warp per
-// block, whose eight heads of q would not fit in registers).
-template <int D, int HPW, int WPB, int NST, int MINB, int SL, bool QSM>
+template <int D, int HPW, int WPB, int NST, int MINB, int SL>
 __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
     attn_splitk_kernel(const AttnParams p) {
   using C = AttnCfg<D, HPW, WPB, NST, SL>;
-  constexpr int OFF_Q = (C::SMEM + 15) / 16 * 16;  // q area (QSM only): [G][QCH][2][8][4] fp32
   extern __shared__ __align__(128) uint8_t smem[];
   uint16_t* stages = reinterpret_cast<uint16_t*>(smem);
   float2* pbuf = reinterpret_cast<float2*>(smem + C::OFF_P);
@@ -426,32 +423,21 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
   griddep_wait();  // q, k_hat, v_hat and the counters are the projection's
   const int hbase = g * C::G + hq * HPW;  // first global q head of this warp
 
-  // q of this lane's key dims, as (even, odd) dim pairs for the packed fp32x2 FMA: in
-  // registers, or (QSM) in shared memory laid out [head][hh][half][dg][4] so that the
-  // eight dg lanes read 128 contiguous bytes
-  float2 q2[QSM ? 1 : HPW][QSM ? 1 : C::QCH][4];
-  float* qsm = reinterpret_cast<float*>(smem + OFF_Q);
-  if constexpr (QSM) {
-    for (int e = threadIdx.x; e < C::G * D; e += C::NCW * 32) {
-      const int h = e / D, d = e % D, c = d / 8, w = d % 8;
-      qsm[(((h * C::QCH + c / 8) * 2 + w / 4) * 8 + c % 8) * 4 + w % 4] =
-          p.qs[((int64_t)b * p.Hq + g * C::G + h) * D + d];
+  // q of this lane's key dims in registers, as (even, odd) dim pairs for the packed
+  // fp32x2 FMA
+  float2 q2[HPW][C::QCH][4];
+#pragma unroll
+  for (int h = 0; h < HPW; ++h)
+#pragma unroll
+    for (int hh = 0; hh < C::QCH; ++hh) {
+      const float4* src = reinterpret_cast<const float4*>(
+          p.qs + ((int64_t)b * p.Hq + hbase + h) * D + (dg + 8 * hh) * 8);
+      const float4 a = src[0], c = src[1];
+      q2[h][hh][0] = make_float2(a.x, a.y);
+      q2[h][hh][1] = make_float2(a.z, a.w);
+      q2[h][hh][2] = make_float2(c.x, c.y);
+      q2[h][hh][3] = make_float2(c.z, c.w);
     }
-    named_bar_sync(1, C::NCW * 32);
-  } else {
-#pragma unroll
-    for (int h = 0; h < HPW; ++h)
-#pragma unroll
-      for (int hh = 0; hh < C::QCH; ++hh) {
-        const float4* src = reinterpret_cast<const float4*>(
-            p.qs + ((int64_t)b * p.Hq + hbase + h) * D + (dg + 8 * hh) * 8);
-        const float4 a = src[0], c = src[1];
-        q2[h][hh][0] = make_float2(a.x, a.y);
-        q2[h][hh][1] = make_float2(a.z, a.w);
-        q2[h][hh][2] = make_float2(c.x, c.y);
-        q2[h][hh][3] = make_float2(c.z, c.w);
-      }
-  }
 
   constexpr int NP = C::DPL / 2;  // value-dim pairs per lane
   float2 acc2[HPW][NP];
@@ -478,38 +464,6 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
       float2 v2[C::NV];
 #pragma unroll
       for (int x = 0; x < C::NV; ++x) v2[x] = make_float2(0.f, 0.f);
-      if constexpr (QSM) {
-        // per 16-byte key chunk: the lane's four tokens unpacked once, then every head's q
-        // read from shared memory (broadcast across the four token groups)
-#pragma unroll
-        for (int hh = 0; hh < C::QCH; ++hh) {
-          float2 kk[4][4];
-#pragma unroll
-          for (int i4 = 0; i4 < 4; ++i4) {
-            const uint4 w = *reinterpret_cast<const uint4*>(Ks + (tg + 4 * i4) * D + (dg + 8 * hh) * 8);
-            kk[i4][0] = make_float2(bf16lo(w.x), bf16hi(w.x));
-            kk[i4][1] = make_float2(bf16lo(w.y), bf16hi(w.y));
-            kk[i4][2] = make_float2(bf16lo(w.z), bf16hi(w.z));
-            kk[i4][3] = make_float2(bf16lo(w.w), bf16hi(w.w));
-          }
-#pragma unroll
-          for (int h = 0; h < HPW; ++h) {
-            const float4* qp = reinterpret_cast<const float4*>(qsm) + (((hq * HPW + h) * C::QCH + hh) * 2) * 8 + dg;
-            const float4 qa = qp[0], qb = qp[8];
-            const float2 q0 = make_float2(qa.x, qa.y), q1 = make_float2(qa.z, qa.w);
-            const float2 q2b = make_float2(qb.x, qb.y), q3 = make_float2(qb.z, qb.w);
-#pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) {
-              float2 a = v2[h * 4 + i4];
-              a = __ffma2_rn(q0, kk[i4][0], a);
-              a = __ffma2_rn(q1, kk[i4][1], a);
-              a = __ffma2_rn(q2b, kk[i4][2], a);
-              a = __ffma2_rn(q3, kk[i4][3], a);
-              v2[h * 4 + i4] = a;
-            }
-          }
-        }
-      } else {
 #pragma unroll
       for (int i4 = 0; i4 < 4; ++i4) {
         const int t = tg + 4 * i4;
@@ -530,7 +484,6 @@ __global__ void __launch_bounds__(AttnCfg<D, HPW, WPB, NST, SL>::THREADS, MINB)
             v2[h * 4 + i4] = a;
           }
         }
-      }
       }
       float v[C::NV];
 #pragma unroll
@@ -942,11 +895,11 @@ static int launch_pdl(void (*fn)(KArgs...), dim3 grid, int threads, int smem, cu
   return cuda_check(cudaLaunchKernelEx(&cfg, fn, std::forward<Args>(args)...), "attention launch");
 }
 
-template <int D, int HPW, int WPB, int NST, int MINB, int SL = kSlots, bool QSM = false>
+template <int D, int HPW, int WPB, int NST, int MINB, int SL = kSlots>
 static int launch_attn_t(const AttnParams& p, int B, int Hkv, cudaStream_t st) {
   using C = AttnCfg<D, HPW, WPB, NST, SL>;
-  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB, SL, QSM>;
-  constexpr int smem = QSM ? (C::SMEM + 15) / 16 * 16 + C::G * D * 4 : C::SMEM;
+  auto* fn = attn_splitk_kernel<D, HPW, WPB, NST, MINB, SL>;
+  constexpr int smem = C::SMEM;
   static bool attr_done = false;  // per instantiation
   if (!attr_done) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1014,11 +967,9 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
       case 1: return launch_attn_t<D, 1, 1, 6, 4, 3>(p, B, Hkv, st);
       case 2: return launch_attn_t<D, 2, 1, 6, 4, 3>(p, B, Hkv, st);
       case 4: return launch_attn_t<D, 4, 1, 6, 4, 3>(p, B, Hkv, st);
-      case 8: return launch_attn_t<D, 4, 2, 6, 2, 3>(p, B, Hkv, st);
+      case 8: return launch_attn_t<D, 4, 2, 4, 3, 2>(p, B, Hkv, st);
     }
   }
-  if (variant == 8 && G == 8) return launch_attn_t<D, 4, 2, 4, 3, 2>(p, B, Hkv, st);
-  if (variant == 9 && G == 8) return launch_attn_t<D, 8, 1, 6, 3, 3, true>(p, B, Hkv, st);
   switch (G) {
     case 1: return launch_attn_t<D, 1, 1, 8, 3>(p, B, Hkv, st);
     case 2: return launch_attn_t<D, 2, 1, 8, 3>(p, B, Hkv, st);
@@ -1031,8 +982,7 @@ static int launch_attn_d(const AttnParams& p, int B, int Hkv, int G, int variant
 int attention_ctas_per_sm(int G, int variant) {
   if (variant == 6) return G == 8 ? 2 : 4;
   if (variant == 7) return G == 8 ? 2 : 3;
-  if ((variant == 8 || variant == 9) && G == 8) return 3;
-  if (variant == 5 || variant == 0) return G == 8 ? 2 : 4;
+  if (variant == 5 || variant == 0) return G == 8 ? 3 : 4;
   return G == 8 ? 1 : 3;
 }
 

@@ -31,17 +31,18 @@ static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant)
   return (29 * slots + 5 * units) / (10 * units);
 }
 
-// The automatic attention kernel (CUDA cores). Four CTAs per SM with three consumer slots
-// (variant 5) beat three CTAs with four slots (variant 1) on long contexts (8B shape,
-// B=16 x 32 K: step 398 vs 411 us, attention alone 354 vs 372 us), but at 2.9 waves of
-// its more numerous CTA slots it cuts short contexts into too many splits (B=4 x 32 K:
-// 54 splits of 38 blocks, 192 vs 147 us per step; both comparisons measured before the
-// split merge was batched). So it is used for G = 4 (the measured group size) when its
-// splits keep at least 100 blocks of the table each; otherwise variant 1.
+// The automatic attention kernel (CUDA cores). Variant 5 packs more CTAs per SM than
+// variant 1: for G = 4 four CTAs of three one-warp slots beat three CTAs of four slots on
+// long contexts (8B shape, B=16 x 32 K: step 398 vs 411 us, attention alone 354 vs 372 us);
+// for G = 8 three CTAs of two two-warp slots beat one CTA of four (70B shape, all blocks
+// in HBM, B=32 x U{8 K..64 K}: 1.20 vs 2.23 ms). At 2.9 waves of its more numerous CTA
+// slots it cuts short contexts into too many splits (B=4 x 32 K, G = 4: 54 splits of 38
+// blocks, 192 vs 147 us per step), so it is used for G = 4 and 8 (the measured group
+// sizes) when its splits keep at least 100 blocks of the table each; otherwise variant 1.
 static int resolve_attn_variant(const dkv_pool* pool, int B, int Hkv, int G, int max_blocks) {
   const int v = pool->tuning.attn_variant;
   if (v != 0) return v;
-  if (G != 4) return 1;
+  if (G != 4 && G != 8) return 1;
   const int s5 = pool->tuning.attn_splits > 0 ? pool->tuning.attn_splits : auto_splits(pool, B, Hkv, G, 5);
   return max_blocks >= 100 * (s5 < 1 ? 1 : s5) ? 5 : 1;
 }

@@ -371,9 +371,11 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
     attr = true;
   }
   const int tiles = a.Hkv * p.nt;
-  // each cluster splits one tile's reduction dimension; about 192 CTAs in total measured
-  // best on B200 for the 8B- and 70B-shaped layers (more CTAs only add reduction work)
-  int CS = a.cluster > 0 ? a.cluster : (192 + tiles / 2) / tiles;
+  // each cluster splits one tile's reduction dimension; about 240 CTAs in total (one wave
+  // at two CTAs per SM) measured best on B200: clusters of 5 for the 8B-shaped layer (48
+  // tiles, 16.9 us vs 18.0 at 4 and 21.0 at 3) and of 3 for the 70B-shaped one (80 tiles,
+  // 41.6 us vs 45.6 at 2 and 51.5 at 5)
+  int CS = a.cluster > 0 ? a.cluster : (240 + tiles / 2) / tiles;
   if (CS < 1) CS = 1;
   if (CS > 8) CS = 8;
   if (CS > p.KB) CS = p.KB;

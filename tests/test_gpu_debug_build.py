@@ -38,7 +38,7 @@ def _cases():
     n = 0
     # decode: layouts, tiers, shapes, group sizes
     for layout in (0, 1):
-        for (Hq, Hkv, D, variants) in ((8, 2, 128, (5, 1, 6)), (16, 2, 128, (5, 1, 8, 9)), (8, 2, 64, (5, 1))):
+        for (Hq, Hkv, D, variants) in ((8, 2, 128, (5, 1, 6)), (16, 2, 128, (5, 1, 6)), (8, 2, 64, (5, 1))):
             cfg = WL.small_config(B=3, Hq=Hq, Hkv=Hkv, D=D, H=256, ctx_range=(1, 400), host_prob=0.5)
             inp = WL.make_decode_inputs(cfg, seed=40 + n, pool_layout=layout)
             ctx = TL.make_pool(inp)
