@@ -260,6 +260,7 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
   const uint16_t* kbase1 = pool.tier[1] + chunk_offset(pool, 1, p.layer, 0, 0, g);
   int pf_tier = 0, pf_phys = 0;
   int issued = 0;
+  const uint64_t kv_policy = l2_policy_evict_first();  // cached KV is read once per step
   // test hook (bounded-wait test): the first CTA never loads nor signals its first block
   const int withheld = (p.withhold && blockIdx.x == 0 && g == 0 && b == 0) ? 0 : -1;
   for (int i = 0; i < n_local; ++i) {
@@ -318,8 +319,8 @@ __device__ __forceinline__ void attn_produce(const AttnParams& p, const CUtensor
             for (int h = 0; h < D / 64; ++h)
               tma_load_2d(dst + kv * CHUNK + h * kT * 128, tmap, 64 * h, row + kv * (int)(kvoff / D), &full[st]);
         } else {
-          bulk_g2s(dst, kp, CHUNK, &full[st]);
-          bulk_g2s(dst + CHUNK, vp, CHUNK, &full[st]);
+          bulk_g2s_hint(dst, kp, CHUNK, &full[st], kv_policy);
+          bulk_g2s_hint(dst + CHUNK, vp, CHUNK, &full[st], kv_policy);
         }
       } else {
         mbar_arrive(&full[st]);

@@ -136,9 +136,13 @@ __global__ void __launch_bounds__(kPThreads, 2)
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // The first ring's W tiles do not depend on the kernel ahead in the stream (weights are
-    // never written by it), so they are fetched before waiting for it; x and everything
-    // after come once it has completed.
+    // W does not depend on the kernel ahead in the stream (weights are never written by
+    // it): the first ring's W tiles are loaded, and the rest of this CTA's W slice is
+    // prefetched into L2, before waiting for it; x and everything after come once it has
+    // completed. (The attention streams its KV with an evict-first L2 policy, so a
+    // projection launched early behind it keeps its prefetched W.)
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
     const int pre = nsteps < nst ? nsteps : nst;
     for (int s = 0; s < pre; ++s) {
       uint8_t* wdst = smem + s * stage_bytes;
@@ -146,6 +150,8 @@ __global__ void __launch_bounds__(kPThreads, 2)
       for (int i = 0; i < np; ++i)
         tma_load_2d(wdst + i * p.D * 128, &tmW, (kb0 + s) * 64, piece_row(p, g, t * p.ppt + i), &full[s]);
     }
+    for (int s = pre; s < nsteps; ++s)
+      for (int i = 0; i < np; ++i) tma_prefetch_l2_2d(&tmW, (kb0 + s) * 64, piece_row(p, g, t * p.ppt + i));
     griddep_wait();
     for (int s = 0; s < pre; ++s) tma_load_2d(smem + s * stage_bytes + kWTile, &tmX, (kb0 + s) * 64, 0, &full[s]);
     for (int s = pre; s < nsteps; ++s) {
