@@ -5,7 +5,9 @@ batch 32, hidden 8192, 64 q / 8 kv heads, head_dim 128, RoPE theta 5e5, cached c
 uniformly from 8192..65536 tokens in 16-token blocks, each block in mapped pinned host memory
 with probability 0.8 (read in place over PCIe) and in HBM otherwise. Its roofline is the host
 link. In the same run the Llama-3-8B-shaped layer with the whole cache in HBM (batch 16,
-32768 cached tokens each) is timed and reported as `hbm_line`, against the HBM roofline. A
+32768 cached tokens each) is timed and reported as `hbm_line`, against the HBM roofline,
+and (one GPU) the remaining configurations — the 8B layer with old blocks in the host tier,
+the tiny layer and the 10240^3 zero-copy GEMM study — as `other_configs`. A
 step is one decode step of one layer through the C ABI (dkv_decode_step: projection,
 split-K attention, combine). Inputs are synthetic (seeded N(0,1) activations and KV,
 W ~ N(0, 1/hidden)), generated on the device.
@@ -49,6 +51,8 @@ def parse():
                     help="decode workload (default: the largest single-GPU configuration; the all-HBM "
                          "8B-shaped layer is then reported beside it as hbm_line)")
     ap.add_argument("--no-hbm-line", action="store_true", help="skip the all-HBM line of the default run")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the 8b_mixed, tiny and GEMM lines of the default run (one GPU)")
     ap.add_argument("--compare-staged", action="store_true",
                     help="host-tier configs: also time swap-in (DMA and copy kernel) + HBM attention")
     ap.add_argument("--attn-splits", type=int, default=0)
@@ -494,13 +498,20 @@ def percentiles(v):
 
 
 def run_gemm(args, rank, world):
-    """The zero-copy GEMM study: C = A . B (10240^3), A in HBM, B in mapped host memory."""
-    import kv_cache_offload_b200 as dkv
+    """The zero-copy GEMM study as its own JSON line (`--config gemm`)."""
     from kv_cache_offload_b200.build import build
     build()
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+    print(json.dumps(gemm_line(args, rank, torch.device("cuda", local))), flush=True)
+
+
+def gemm_line(args, rank, dev, steps=None, warmup=None):
+    """The zero-copy GEMM study: C = A . B (10240^3), A in HBM, B in mapped host memory;
+    CPU-aware tiling, naive zero-copy, staged swap and both operands in HBM."""
+    import kv_cache_offload_b200 as dkv
+    steps = steps or args.steps
+    warmup = warmup or args.warmup
     cfg = WL.GEMM_CONFIGS["gemm"]
     M, N, K = cfg.M, cfg.N, cfg.K
     if args.gemm_dim:
@@ -515,28 +526,29 @@ def run_gemm(args, rank, world):
     res = {}
     flops = 2.0 * M * N * K
     b_bytes = N * K * 2
-    for name, steps in (("DEVICE", args.steps), ("CPU_AWARE", args.steps), ("STAGED_SWAP", args.steps),
-                        ("NAIVE_ZERO_COPY", max(1, min(args.steps, 3)))):
+    for name, n in (("DEVICE", steps), ("CPU_AWARE", steps), ("STAGED_SWAP", steps),
+                    ("NAIVE_ZERO_COPY", max(1, min(steps, 3)))):
         v = getattr(dkv, "DKV_GEMM_" + name)
         ws = torch.empty(dkv.dkv_gemm_workspace_bytes(v, M, N, K), dtype=torch.uint8, device=dev)
         b = Btd if name == "DEVICE" else hb.dev_ptr
-        for _ in range(1 if name == "NAIVE_ZERO_COPY" else args.warmup):
+        for _ in range(1 if name == "NAIVE_ZERO_COPY" else warmup):
             dkv.dkv_gemm(v, A, b, C, ws, M, N, K)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for _ in range(steps):
+        for _ in range(n):
             dkv.dkv_gemm(v, A, b, C, ws, M, N, K)
         e1.record()
         e1.synchronize()
-        ms = e0.elapsed_time(e1) / steps
+        ms = e0.elapsed_time(e1) / n
         res[name] = {"ms": ms, "tflops": flops / (ms * 1e-3) / 1e12}
         del ws
     h2d = measure_h2d_peak(dev)
     hb.close()
     ca = res["CPU_AWARE"]["ms"]
+    del A, Btd, C
     line = {"metric": "zero-copy GEMM 10240^3 time (CPU-aware tiling)", "value": ca, "unit": "ms",
-            "higher_is_better": False, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": False, "n_gpus": 1, "steps": steps, "warmup": warmup,
             "dtype": "bf16", "data": "synthetic", "impl": "dkv",
             "config": {"workload": "gemm: C = A.B, M=N=K=%d, A bf16 in HBM, B bf16 column-major in mapped "
                                    "pinned host memory, fp32 accumulate/output" % M},
@@ -547,7 +559,7 @@ def run_gemm(args, rank, world):
                           "naive_model_host_bytes_BM128": (M // 128) * b_bytes,
                           "link": "PCIe (not NVLink-C2C)"},
             "pages_context": {"swap_ms": 65, "naive_ms": 1122, "hardware": "PCIe platform, GPU unstated"}}
-    print(json.dumps(line), flush=True)
+    return line
 
 
 def run_layout(args):
@@ -808,6 +820,7 @@ def run_adaptive(args):
 
 HEADLINE = "70b_mixed"  # the largest single-GPU decode configuration: the headline line
 HBM_LINE = "8b_hbm"     # the all-HBM configuration, reported beside it in the same run
+OTHER_CONFIGS = ("8b_mixed", "tiny")  # the remaining decode configurations (with the GEMM study)
 
 
 def _nvtx(name):
@@ -1101,6 +1114,21 @@ def main():
         hl = decode_line(WL.CONFIGS[HBM_LINE], args, world, rank, local, dist, dev, full=False, steps=hsteps)
         hl.update(unit="tokens/s", steps=hsteps)
         line["hbm_line"] = hl
+    if args.config == HEADLINE and not args.batch and not args.ctx and world == 1 and not args.no_other_configs:
+        # the remaining decode configurations and the GEMM study, in the same run (one GPU)
+        torch.cuda.empty_cache()
+        other = {}
+        for name in OTHER_CONFIGS:
+            # the 8B mixed layer also runs the conventional offload on the same workload: swap
+            # the host blocks into HBM (per-block DMA or the GPU copy kernel), then attend
+            args.compare_staged = name == "8b_mixed"
+            o = decode_line(WL.CONFIGS[name], args, world, rank, local, dist, dev, full=False,
+                            steps=min(args.steps, 20))
+            o.update(unit="tokens/s", steps=min(args.steps, 20))
+            other[name] = o
+            torch.cuda.empty_cache()
+        other["gemm"] = gemm_line(args, rank, dev, steps=min(args.steps, 5), warmup=3)
+        line["other_configs"] = other
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, 0, args.cpu_seconds)
     if rank == 0:
