@@ -285,8 +285,9 @@ size_t dkv_decode_static_workspace_capacity(void);
 int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 
 /* The attention kernel variant dkv_decode_step runs for this shape: the pool's
- * dkv_tuning.attn_variant, or, when that is 0, the automatic choice (for Hq/Hkv = 4 or 8: 5
- * when its split-K ranges keep at least 100 blocks of the table each, else 1; 1 otherwise).
+ * dkv_tuning.attn_variant, or, when that is 0, the automatic choice (Hq/Hkv = 4: 5 when its
+ * split-K ranges keep at least 39 blocks of the table each, else 1; Hq/Hkv = 8: 5 when they
+ * keep at least 6 blocks and there are at most 64 of them, else 1; other group sizes: 1).
  * Returns the variant (> 0) or a negative DKV_ERR_* code. */
 int dkv_decode_attn_variant(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 

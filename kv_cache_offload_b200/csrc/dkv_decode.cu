@@ -31,20 +31,26 @@ static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant)
   return (29 * slots + 5 * units) / (10 * units);
 }
 
-// The automatic attention kernel (CUDA cores). Variant 5 packs more CTAs per SM than
-// variant 1: for G = 4 four CTAs of three one-warp slots beat three CTAs of four slots on
-// long contexts (8B shape, B=16 x 32 K: step 398 vs 411 us, attention alone 354 vs 372 us);
-// for G = 8 three CTAs of two two-warp slots beat one CTA of four (70B shape, all blocks
-// in HBM, B=32 x U{8 K..64 K}: 1.20 vs 2.23 ms). At 2.9 waves of its more numerous CTA
-// slots it cuts short contexts into too many splits (B=4 x 32 K, G = 4: 54 splits of 38
-// blocks, 192 vs 147 us per step), so it is used for G = 4 and 8 (the measured group
-// sizes) when its splits keep at least 100 blocks of the table each; otherwise variant 1.
+// The automatic attention kernel (CUDA cores): variant 5 packs more CTAs per SM than
+// variant 1 (G = 4: four CTAs of three one-warp slots vs three of four slots; G = 8: three
+// CTAs of two two-warp slots vs one of four), which streams long contexts faster, but at
+// 2.9 waves of its more numerous CTA slots it cuts short contexts into more, shorter splits.
+// Measured on B200 (attention alone, all blocks in HBM, B in {1, 4, 8, 16, 32} x {2 K, 8 K,
+// 32 K} tokens, automatic split counts): G = 4 takes variant 5 once its splits keep at
+// least 39 blocks of the table each (B=16 x 32 K: 353 vs 375 us; B=8 x 32 K: 190 vs 202;
+// B=32 x 8 K: 198 vs 205; B=4 x 32 K at 38 blocks: 118 vs 117); G = 8 takes it once its
+// splits keep at least 6 blocks and there are at most 64 of them (B=8 x 32 K: 304 vs 584
+// us; B=32 x 2 K: 100 vs 154; B=8 x 2 K at 6.5 blocks: 49 vs 60; a single sequence, 129-161
+// splits: 55-96 vs 33-84). Other group sizes: variant 1.
 static int resolve_attn_variant(const dkv_pool* pool, int B, int Hkv, int G, int max_blocks) {
   const int v = pool->tuning.attn_variant;
   if (v != 0) return v;
   if (G != 4 && G != 8) return 1;
-  const int s5 = pool->tuning.attn_splits > 0 ? pool->tuning.attn_splits : auto_splits(pool, B, Hkv, G, 5);
-  return max_blocks >= 100 * (s5 < 1 ? 1 : s5) ? 5 : 1;
+  int s5 = pool->tuning.attn_splits > 0 ? pool->tuning.attn_splits : auto_splits(pool, B, Hkv, G, 5);
+  if (s5 < 1) s5 = 1;
+  const int blocks_per_split = max_blocks / s5;
+  if (G == 4) return blocks_per_split >= 39 ? 5 : 1;
+  return blocks_per_split >= 6 && s5 <= 64 ? 5 : 1;
 }
 
 static int pick_attn_splits(const dkv_pool* pool, int B, int Hkv, int G, int max_blocks) {
