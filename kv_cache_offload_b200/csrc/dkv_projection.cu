@@ -16,11 +16,11 @@
 //  * While W streams, the otherwise idle warps look up, for every batch column b the CTA
 //    will finish (b = r, r + CS, ... for cluster rank r), its position and cache-slot
 //    addresses, and compute the RoPE (cos, sin) of each rotation pair at that position.
-//  * Each CTA then reads its partial [128 x N] accumulator from TMEM and stores column b
-//    straight into the shared memory of the CTA that finishes it (distributed shared
-//    memory, rank b mod CS); after one cluster barrier every CTA sums its columns over the
-//    CS partials in rank order from its own shared memory (a fixed order: deterministic)
-//    and finishes them: q heads rotated and scaled by log2(e)/sqrt(D) for the log2-domain
+//  * Each CTA then copies its partial [128 x N] accumulator from TMEM into its own shared
+//    memory; after one cluster barrier the CTA of rank r reads columns b = r, r + CS, ...
+//    from all CS partials (distributed shared memory; independent loads, issued together)
+//    and sums them in rank order (a fixed order: deterministic). It then finishes them:
+//    q heads rotated and scaled by log2(e)/sqrt(D) for the log2-domain
 //    softmax, the key head rotated and rounded to bf16 (k_hat), the value head rounded
 //    (v_hat); k_hat and v_hat are written once into the cache slot and, as fp32, into the
 //    workspace for the new token's attention term.
@@ -51,7 +51,8 @@ struct ProjParams {
   int B, H, Hq, Hkv, D, G;
   int ppt, nt, Npad, CS, KB, nst;
   int slots;                           // batch columns a CTA finishes: ceil(B / CS)
-  int off_recv, off_rope, off_cols, off_bars;  // shared-memory carve-up (bytes)
+  int pdl;                             // launched with programmatic dependent launch
+  int off_part, off_rope, off_cols, off_bars;  // shared-memory carve-up (bytes)
   float qscale;
   float* qs;              // [B][Hq][D]
   float* knew;            // [B][Hkv][D]
@@ -60,15 +61,13 @@ struct ProjParams {
   double inv_freq[64];    // theta^(-2i/D), i < D/2, computed on the host in fp64
 };
 
-// Distributed-shared-memory access: address of `p` in CTA `rank` of the cluster, and a
-// 32-bit store through that address.
-__device__ __forceinline__ uint32_t dsmem_map(const void* p, int rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
-  return r;
+// Split cluster barrier: arrive (releasing this thread's prior memory operations) and wait
+// (acquiring the other CTAs' released ones); every thread of every CTA takes both.
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void dsmem_st(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Epilogue lookups done while W streams, one per batch column the CTA finishes: the
@@ -79,6 +78,35 @@ struct EpiCol {
   int pos;
   int pad;
 };
+
+// Sum, for each column b = rank + CS * it (it < slots, b < B) this CTA finishes, row `row`
+// of the CS partial accumulators part[b][128] held by the cluster's CTAs, in rank order,
+// into colsum[it][row]. Columns go in groups of 8, each group's 8 x CS remote reads issued
+// together.
+template <int CS>
+__device__ __forceinline__ void pull_columns(cg::cluster_group& cluster, float* part, float* colsum, int rank,
+                                             int slots, int B, int row) {
+  const float* peer[CS];
+#pragma unroll
+  for (int q = 0; q < CS; ++q) peer[q] = cluster.map_shared_rank(part, q);
+  for (int it0 = 0; it0 < slots; it0 += 8) {
+    float v[8][CS];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int b = rank + CS * (it0 + i);
+      const bool ok = it0 + i < slots && b < B;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) v[i][q] = ok ? peer[q][b * 128 + row] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float x = 0.f;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) x += v[i][q];
+      if (it0 + i < slots) colsum[(it0 + i) * 128 + row] = x;
+    }
+  }
+}
 
 // First W row of piece (head) `pc` of kv-head group g: pieces 0..G-1 are the group's q
 // heads, G its key head, G+1 its value head.
@@ -98,7 +126,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
   const int g = tile / p.nt, t = tile % p.nt;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // 1024-byte aligned carve-up: ring | column receive area | RoPE table | column lookups |
+  // 1024-byte aligned carve-up: ring | partial accumulator | RoPE table | column lookups |
   // barriers | tmem slot
   const uint32_t base_u = smem_u32(psmem_raw);
   uint8_t* smem = psmem_raw + (((base_u + 1023u) & ~1023u) - base_u);
@@ -106,7 +134,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
   const int stage_bytes = kWTile + xtile;
   const int nst = p.nst;
   const int slots = p.slots;
-  float* recv = reinterpret_cast<float*>(smem + p.off_recv);     // [CS][slots][128] partial columns
+  float* part = reinterpret_cast<float*>(smem + p.off_part);     // [B][128] this CTA's partial
   float2* rope = reinterpret_cast<float2*>(smem + p.off_rope);   // [slots][D/2] (cos, sin)
   EpiCol* cols = reinterpret_cast<EpiCol*>(smem + p.off_cols);   // [slots]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.off_bars);
@@ -114,7 +142,10 @@ __global__ void __launch_bounds__(kPThreads, 2)
   uint64_t* done = empty + nst;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
 
-  if (tid == 0) {
+  // TMEM first: a second CTA is placed on this SM only once this one has given up its
+  // allocation permit (tmem_alloc relinquishes it), so the allocation leads the prologue
+  if (warp == 0) tmem_alloc(tmem_slot, 32);
+  if (tid == 32) {
     for (int i = 0; i < nst; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
@@ -122,7 +153,6 @@ __global__ void __launch_bounds__(kPThreads, 2)
     mbar_init(done, 1);
     mbar_fence_init();
   }
-  if (warp == 0) tmem_alloc(tmem_slot, 32);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -150,8 +180,9 @@ __global__ void __launch_bounds__(kPThreads, 2)
       for (int i = 0; i < np; ++i)
         tma_load_2d(wdst + i * p.D * 128, &tmW, (kb0 + s) * 64, piece_row(p, g, t * p.ppt + i), &full[s]);
     }
-    for (int s = pre; s < nsteps; ++s)
-      for (int i = 0; i < np; ++i) tma_prefetch_l2_2d(&tmW, (kb0 + s) * 64, piece_row(p, g, t * p.ppt + i));
+    if (p.pdl)  // only worth its issue cost (~0.1 us each) when there is a kernel to overlap
+      for (int s = pre; s < nsteps; ++s)
+        for (int i = 0; i < np; ++i) tma_prefetch_l2_2d(&tmW, (kb0 + s) * 64, piece_row(p, g, t * p.ppt + i));
     griddep_wait();
     for (int s = 0; s < pre; ++s) tma_load_2d(smem + s * stage_bytes + kWTile, &tmX, (kb0 + s) * 64, 0, &full[s]);
     for (int s = pre; s < nsteps; ++s) {
@@ -238,24 +269,19 @@ __global__ void __launch_bounds__(kPThreads, 2)
   __syncwarp();
   griddep_wait();
 
-  // -------------------------------- TMEM -> the shared memory of each column's finisher
-  // column b goes to cluster rank b mod CS, slot b / CS, as its row-`tid` element
+  // ------------------------------------ partial accumulator: TMEM -> own shared memory
   mbar_wait_bounded(done, 0, p.pool.status);
   tc_fence_after();
   for (int c0 = 0; c0 < p.Npad; c0 += 16) {
     float v[16];
     tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int b = c0 + j;
-      if (b < p.B)
-        dsmem_st(dsmem_map(recv + ((size_t)(rank * slots + b / p.CS) * 128 + tid), b % p.CS), v[j]);
-    }
+    for (int j = 0; j < 16; ++j)
+      if (c0 + j < p.B) part[(c0 + j) * 128 + tid] = v[j];
   }
   tc_fence_before();
   if (t == 0 && rank == 0 && tid < p.B && p.attn_cnt) p.attn_cnt[(int64_t)tid * p.Hkv + g] = 0;
-  cluster.sync();  // every partial column has arrived where it is finished (and no CTA
-                   // touches another's shared memory after this)
+  cluster.sync();  // every CTA's partial is in its shared memory
   tc_fence_after();
   if (warp == 0) tmem_dealloc(tmem, 32);
 
@@ -268,11 +294,28 @@ __global__ void __launch_bounds__(kPThreads, 2)
   const int pc = t * p.ppt + row / D;     // piece (head) index within the group
   const int d = row % D, pi = d % half;   // RoPE pair index
   const bool live = row / D < np;
+  // column b is finished by cluster rank b mod CS: it reads row `row` of column b from the
+  // CS partials (peers' shared memory) and sums them in rank order (deterministic). A
+  // remote read costs about a microsecond of latency, so all of a thread's reads (up to 8
+  // columns x CS ranks) are issued before the first sum; the sums go to the ring, free
+  // once the MMAs have completed.
+  float* colsum = reinterpret_cast<float*>(smem);  // [slots][128]
+  switch (p.CS) {
+    case 1: pull_columns<1>(cluster, part, colsum, rank, slots, p.B, row); break;
+    case 2: pull_columns<2>(cluster, part, colsum, rank, slots, p.B, row); break;
+    case 3: pull_columns<3>(cluster, part, colsum, rank, slots, p.B, row); break;
+    case 4: pull_columns<4>(cluster, part, colsum, rank, slots, p.B, row); break;
+    case 5: pull_columns<5>(cluster, part, colsum, rank, slots, p.B, row); break;
+    case 6: pull_columns<6>(cluster, part, colsum, rank, slots, p.B, row); break;
+    case 7: pull_columns<7>(cluster, part, colsum, rank, slots, p.B, row); break;
+    default: pull_columns<8>(cluster, part, colsum, rank, slots, p.B, row); break;
+  }
+  cluster_arrive_release();  // done with the peers' shared memory
+
   for (int it = 0; it < slots; ++it) {
     const int b = rank + p.CS * it;
     if (b >= p.B) break;
-    float x = 0.f;
-    for (int q = 0; q < p.CS; ++q) x += recv[(q * slots + it) * 128 + row];  // rank order: deterministic
+    float x = colsum[it * 128 + row];  // written by this thread above
     const float xp = __shfl_xor_sync(0xffffffffu, x, 16);  // the pair's other row
     if (!live) continue;
     if (pc <= p.G) {
@@ -292,6 +335,7 @@ __global__ void __launch_bounds__(kPThreads, 2)
     uint16_t* dst = cols[it].dst[kv];
     if (dst) dst[d] = hb;
   }
+  cluster_wait_acquire();  // no CTA leaves while a peer may still read its partial
 }
 
 // ------------------------------------------------------------------ host side
@@ -331,8 +375,8 @@ constexpr int kProjSmemBudget = 113 * 1024;
 static int proj_smem_layout(ProjParams* p, int nst) {
   const int stage = kWTile + p->Npad * 128;
   int o = nst * stage;
-  p->off_recv = o;
-  o += p->CS * p->slots * 128 * 4;
+  p->off_part = o;
+  o += p->B * 128 * 4;
   p->off_rope = o;
   o += p->slots * (p->D / 2) * 8;
   p->off_cols = o;
@@ -359,6 +403,7 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
   p.KB = a.H / 64;
   for (int i = 0; i < a.D / 2; ++i) p.inv_freq[i] = pow(a.theta, -2.0 * (double)i / (double)a.D);
   p.attn_cnt = a.attn_cnt;
+  p.pdl = a.pdl;
   p.qscale = a.qscale;
   p.qs = a.qs;
   p.knew = a.knew;
