@@ -10,7 +10,8 @@ and (one GPU) the remaining configurations — the 8B layer with old blocks in t
 the tiny layer and the 10240^3 zero-copy GEMM study — as `other_configs`. A
 step is one decode step of one layer through the C ABI (dkv_decode_step: projection,
 split-K attention, combine). Inputs are synthetic (seeded N(0,1) activations and KV,
-W ~ N(0, 1/hidden)), generated on the device.
+W ~ N(0, 1/hidden)), generated on the device; steps cycle through several copies of W
+(more than twice the L2 in all), as a model's layers would, so W is read from HBM.
 
 Multi-GPU: every rank runs an independent replica of the workload (the step has no
 cross-GPU exchange); value = tokens of all ranks / max-over-ranks time. Each rank's host
@@ -107,6 +108,22 @@ def profiled_traffic(config_name: str, batch: int):
     if e.get("batch") != batch:
         return None
     return {"bytes": e.get("bytes_per_launch"), "counter": e.get("counter")}
+
+
+_NVML = {}
+
+
+def sm_clock_now(index: int):
+    """The GPU's SM clock (MHz) read through NVML at this moment, or None without NVML."""
+    try:
+        import pynvml
+        if "h" not in _NVML:
+            pynvml.nvmlInit()
+            _NVML["h"] = {}
+        h = _NVML["h"].setdefault(index, pynvml.nvmlDeviceGetHandleByIndex(index))
+        return pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+    except Exception:
+        return None
 
 
 class ClockSampler:
@@ -219,7 +236,14 @@ class Workload:
                 e = min(n, s + step)
                 host[s:e].copy_(gpu_randn_bf16((e - s,), gen).view(torch.int16).cpu())
         self.x = gpu_randn_bf16((cfg.B, cfg.H), gen)
-        self.W = gpu_randn_bf16((cfg.rows, cfg.H), gen, std=1.0 / math.sqrt(cfg.H))
+        # one W per layer, as in a model: steps cycle through enough copies (more than twice
+        # the L2 in all) that no step finds its W left in L2 by an earlier one — a model uses
+        # a layer's W again only a whole forward pass later
+        self.w_bytes = cfg.rows * cfg.H * 2
+        l2 = getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20)
+        self.n_w = min(8, max(1, math.ceil(2 * l2 / self.w_bytes)))
+        self.Ws = [gpu_randn_bf16((cfg.rows, cfg.H), gen, std=1.0 / math.sqrt(cfg.H)) for _ in range(self.n_w)]
+        self.k_w = 0
         self.table = lay.block_table.to(dev)
         self.tmap = lay.tier_map.to(dev)
         self.lens = torch.tensor(lay.seq_lens, dtype=torch.int32, device=dev)
@@ -239,7 +263,6 @@ class Workload:
         self.kv_host_bytes = host_tok * per_tok
         self.kv_hbm_bytes = hbm_tok * per_tok
         self.kv_bytes = self.kv_host_bytes + self.kv_hbm_bytes
-        self.w_bytes = cfg.rows * cfg.H * 2
         self.new_kv_bytes = cfg.B * cfg.Hkv * cfg.D * 2 * 2
         self.splits = dkv.dkv_decode_attn_splits(self.pool, cfg.B, lay.max_blocks, cfg.Hq)
 
@@ -252,16 +275,31 @@ class Workload:
             self.nws = n
             self.ws = torch.empty(n, dtype=torch.uint8, device=self.ws.device)
 
+    @property
+    def W(self):
+        """The next step's W (advanced by next_W)."""
+        return self.Ws[self.k_w % self.n_w]
+
+    def next_W(self):
+        W = self.W
+        self.k_w += 1
+        return W
+
     def step(self):
         c = self.cfg
-        self.dkv.dkv_decode_step(self.pool, 0, self.x, self.W, self.table, self.lens, self.tmap, c.Hq,
+        self.dkv.dkv_decode_step(self.pool, 0, self.x, self.next_W(), self.table, self.lens, self.tmap, c.Hq,
                                  c.theta, self.out, self.ws)
+
+    def project(self):
+        c = self.cfg
+        self.dkv.dkv_decode_project(self.pool, 0, self.x, self.next_W(), self.table, self.lens, self.tmap, c.Hq,
+                                    c.theta, self.ws)
 
     def step_timed_stages(self, ev):
         """The same step as step(), with events between its two launches."""
         c, d = self.cfg, self.dkv
         ev[0].record()
-        d.dkv_decode_project(self.pool, 0, self.x, self.W, self.table, self.lens, self.tmap, c.Hq,
+        d.dkv_decode_project(self.pool, 0, self.x, self.next_W(), self.table, self.lens, self.tmap, c.Hq,
                              c.theta, self.ws)
         ev[1].record()
         d.dkv_decode_attend(self.pool, 0, self.table, self.lens, self.tmap, c.H, c.Hq, self.ws,
@@ -642,7 +680,7 @@ def run_staged_compare(args, cfg, wl, dev):
 
             def step():
                 dkv.dkv_copy_blocks(pool, 1, 0, s_ids, d_ids, method)
-                dkv.dkv_decode_step(pool, 0, wl.x, wl.W, table, wl.lens, tmap, cfg.Hq, cfg.theta, wl.out, wl.ws)
+                dkv.dkv_decode_step(pool, 0, wl.x, wl.next_W(), table, wl.lens, tmap, cfg.Hq, cfg.theta, wl.out, wl.ws)
 
             step()
             torch.cuda.synchronize()
@@ -873,6 +911,7 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
             wl.step()
         e1.record()
         barrier()
+        pass_mhz = {"timed": sm_clock_now(local)}
         _nvtx_end()
         time.sleep(0.25)
         clk = clocks.stop()
@@ -889,6 +928,7 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
             wl.step()
             evs[i + 1].record()
         barrier()
+        pass_mhz["per_step"] = sm_clock_now(local)
         _nvtx_end()
         per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
 
@@ -903,8 +943,25 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
         for i in range(steps):
             wl.step_timed_stages(sevs[i])
         barrier()
+        pass_mhz["stages"] = sm_clock_now(local)
         stage_ms = [sum(sevs[i][k].elapsed_time(sevs[i][k + 1]) for i in range(steps)) / steps
                     for k in range(2)]
+        # ---- the projection alone, back to back: serial launches queued while a sleep kernel
+        # holds the stream, timed between two events. Its GPU time per launch, including the
+        # gap every kernel launch costs (~2 us on each side here) but not the two events per
+        # stage above; W cycles through its copies, so it comes from HBM.
+        n_proj = 100
+        for _ in range(3):
+            wl.project()
+        barrier()
+        torch.cuda._sleep(10_000_000)  # a few ms at the SM clock: the host queues the launches meanwhile
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record()
+        for _ in range(n_proj):
+            wl.project()
+        p1.record()
+        barrier()
+        proj_b2b_ms = p0.elapsed_time(p1) / n_proj
         wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant)
         _nvtx_end()
 
@@ -916,9 +973,9 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
 
         # ---- max over ranks
         p10, p50, p90 = percentiles(per_step)
-        vals = reduce_max_over_ranks([t_ms, e2e_ms, p10, p50, p90] + stage_ms, dist, dev)
-        t_ms, e2e_ms, p10, p50, p90 = vals[:5]
-        stage_ms = vals[5:]
+        vals = reduce_max_over_ranks([t_ms, e2e_ms, p10, p50, p90, proj_b2b_ms] + stage_ms, dist, dev)
+        t_ms, e2e_ms, p10, p50, p90, proj_b2b_ms = vals[:6]
+        stage_ms = vals[6:]
         ms = t_ms / steps
         value = replica_throughput(cfg.B, world, ms)
 
@@ -942,13 +999,22 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
             "step_ms_p10_p50_p90": [p10, p50, p90],
             "config": dict(workload_config(cfg, world), attn_splits=wl.splits, attn_variant=args.attn_variant,
                            attn_kernel_variant=dkv.dkv_decode_attn_variant(wl.pool, cfg.B, wl.lay.max_blocks, cfg.Hq),
-                           l2="inputs larger than L2 (%.2f GB of KV + W per step)" % ((wl.kv_bytes + wl.w_bytes) / 1e9)),
+                           l2="inputs larger than L2 (%.2f GB of KV + W per step; W cycles through %d copies, "
+                              "%.2f GB)" % ((wl.kv_bytes + wl.w_bytes) / 1e9, wl.n_w, wl.n_w * wl.w_bytes / 1e9)),
             "kv_gbs": (wl.kv_bytes + wl.new_kv_bytes) / (ms * 1e-3) / 1e9,
             # the whole step against the same peak: every byte it must move (cached KV, W, x,
             # the new K/V rows, out) over the step time (host-tier bytes over the host link)
             "step_roofline": step_roofline(wl, ms, peak, peak_kind),
             "stage_ms": {"project": stage_ms[0], "attend_and_combine": stage_ms[1],
-                         "timing": "each kernel alone (serial launches); the step overlaps them"},
+                         "timing": "each kernel alone (serial launches) between events; the step overlaps them",
+                         "project_back_to_back": proj_b2b_ms,
+                         "project_back_to_back_timing": "%d serial launches queued behind a sleep kernel, "
+                                                        "between two events, W from HBM" % n_proj},
+            "projection_roofline": {"bound": "hbm", "kernel": "proj_umma_kernel",
+                                    "achieved": wl.w_bytes / (proj_b2b_ms * 1e-3) / 1e9, "peak": peak,
+                                    "unit": "GB/s", "frac": wl.w_bytes / (proj_b2b_ms * 1e-3) / 1e9 / peak,
+                                    "peak_source": peak_kind, "algorithmic_bytes_per_launch": wl.w_bytes,
+                                    "timing": "stage_ms.project_back_to_back"},
             "roofline": ({"bound": "hbm", "kernel": "attn_splitk_kernel",
                           "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                           "peak_source": peak_kind, "traffic": tr and tr["bytes"],
@@ -963,6 +1029,9 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
                           "algorithmic_bytes_per_launch": wl.kv_host_bytes}),
             "gpu_launches": 2 * steps,
             "clocks": clk,
+            # SM clock (NVML) at the end of each pass: the power-capped clock differs from pass
+            # to pass, and the step and stage times follow it
+            "pass_end_sm_mhz": pass_mhz,
         }
         if full:
             line["e2e"] = {"value": replica_throughput(cfg.B, world, e2e_ms / steps), "unit": "tokens/s",
@@ -1012,7 +1081,7 @@ def time_e2e(wl, steps, barrier):
         i = k % 2
         xd, td, md, ld = ins[i]
         main.wait_event(ev_in[i])
-        dkv.dkv_decode_step(wl.pool, 0, xd, wl.W, td, ld, md, cfg.Hq, cfg.theta, outs[i], wl.ws)
+        dkv.dkv_decode_step(wl.pool, 0, xd, wl.next_W(), td, ld, md, cfg.Hq, cfg.theta, outs[i], wl.ws)
         ev_done[i].record(main)
         # copy stream, while step k computes: read back step k-1's output, then refill that
         # buffer set with step k+1's inputs (step k+1 waits for them, hence for the read-back)
