@@ -51,6 +51,24 @@ def test_ragged_lengths_both_tiers_both_layouts(layout):
     _run_and_check(cfg, layout=layout, layer=1, seq_lens=[0, 1, 15, 16, 17, 100, 257])
 
 
+@pytest.mark.parametrize("cs", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("B", [3, 13, 32])
+def test_projection_cluster_sizes(cs, B):
+    """Every cluster size of the projection's split-K reduction (its gather of the partial
+    columns is compiled per size), with batches below, between and at multiples of it
+    (B < CS leaves ranks that finish no column)."""
+    cfg = WL.small_config(B=B, H=512, ctx_range=(1, 64))
+    inp = WL.make_decode_inputs(cfg, seed=cs)
+    ctx = TL.make_pool(inp)
+    try:
+        out = TL.run_step(ctx, layer=1, proj_splits=cs)
+        ores = TL.oracle_step(inp, layer=1)
+        TL.assert_out_close(out, ores["out"], cfg.name)
+        TL.check_cache(ctx, ores, layer=1)
+    finally:
+        ctx.close()
+
+
 @pytest.mark.parametrize("splits", [1, 2, 5, 64])
 def test_split_counts(splits):
     cfg = WL.small_config(B=2, ctx_range=(300, 400))
