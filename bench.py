@@ -48,7 +48,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="dkv", choices=["dkv", "reference"])
-    ap.add_argument("--config", default="70b_mixed", choices=sorted(WL.CONFIGS) + ["gemm", "layout", "adaptive"],
+    ap.add_argument("--config", default="70b_mixed",
+                    choices=sorted(WL.CONFIGS) + ["gemm", "layout", "adaptive", "host_contention"],
                     help="decode workload (default: the largest single-GPU configuration; the all-HBM "
                          "8B-shaped layer is then reported beside it as hbm_line)")
     ap.add_argument("--no-hbm-line", action="store_true", help="skip the all-HBM line of the default run")
@@ -800,6 +801,80 @@ class AdaptiveModel:
         self.dkv.dkv_pool_destroy(self.pool)
 
 
+def _dram_reader(nbytes, stop, counter, ready):
+    """Another consumer of host DRAM bandwidth: streams through a private buffer until
+    `stop` is set, adding the bytes read to `counter`."""
+    import numpy as np
+    a = np.ones(nbytes // 8, dtype=np.float64)  # touched, so resident
+    ready.put(1)
+    while not stop.is_set():
+        a.max()
+        with counter.get_lock():
+            counter.value += nbytes
+
+
+def run_host_contention(args):
+    """NEXT-4 on one GPU: the host-tier decode step of the 70B-shaped layer (80% of its
+    blocks read in place over PCIe) while k spawned CPU processes stream through their own
+    host buffers, standing in for the host-DRAM traffic of other GPUs' replicas. Per k: the
+    step's host-tier read rate, the readers' aggregate rate, and cudaMemcpy H2D under the
+    same load."""
+    import multiprocessing as mp
+    import kv_cache_offload_b200 as dkv
+    from kv_cache_offload_b200.build import build
+    build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg = WL.CONFIGS["70b_mixed"]
+    wl = Workload(cfg, seed=0, host_flags=args.host_flags)
+    ctx = mp.get_context("spawn")  # never fork a process that has a CUDA context
+    steps = max(3, min(args.steps, 8))
+    sweep = []
+    try:
+        for _ in range(max(3, args.warmup)):
+            wl.step()
+        torch.cuda.synchronize()
+        for k in (0, 2, 4, 8, 12):
+            stop, counter, ready = ctx.Event(), ctx.Value("d", 0.0), ctx.Queue()
+            procs = [ctx.Process(target=_dram_reader, args=(512 << 20, stop, counter, ready), daemon=True)
+                     for _ in range(k)]
+            for pr in procs:
+                pr.start()
+            try:
+                for _ in procs:
+                    ready.get(timeout=120)
+                time.sleep(0.5)
+                c0, t0 = counter.value, time.perf_counter()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                for _ in range(steps):
+                    wl.step()
+                b.record()
+                b.synchronize()
+                c1, t1 = counter.value, time.perf_counter()
+                ms = a.elapsed_time(b) / steps
+                h2d = measure_h2d_peak(dev, nbytes=512 << 20, reps=3)
+            finally:
+                stop.set()
+                for pr in procs:
+                    pr.join(timeout=30)
+            assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
+            sweep.append({"readers": k, "ms_per_step": ms, "tokens_per_s": cfg.B / (ms * 1e-3),
+                          "host_tier_gbs": wl.kv_host_bytes / (ms * 1e-3) / 1e9,
+                          "readers_gbs": (c1 - c0) / (t1 - t0) / 1e9, "h2d_memcpy_gbs": h2d})
+    finally:
+        wl.close()
+    base = sweep[0]["host_tier_gbs"]
+    line = {"metric": "host-tier zero-copy read rate under host-DRAM contention (70B-shaped layer)",
+            "value": sweep[-1]["host_tier_gbs"], "unit": "GB/s", "n_gpus": 1, "higher_is_better": True,
+            "config": {"workload": workload_config(cfg, 1)["workload"], "steps_per_point": steps,
+                       "readers": "spawned CPU processes, each streaming a private 512 MiB buffer (max reduction)",
+                       "host_cpus": os.cpu_count()},
+            "sweep": sweep, "retained_at_max_readers": sweep[-1]["host_tier_gbs"] / base,
+            "note": "the host-tier rate is over the whole step (projection + attention)"}
+    print(json.dumps(line), flush=True)
+
+
 def run_adaptive(args):
     """Adaptive placement (hot blocks in HBM, cold blocks read in place from the host tier)
     over a 4-layer slice of the 8B-shaped model, B=16 x 32768 cached tokens (8 GiB of KV),
@@ -1116,6 +1191,8 @@ def main():
         return run_layout(args)
     if args.config == "adaptive":
         return run_adaptive(args)
+    if args.config == "host_contention":
+        return run_host_contention(args)
     if args.config == "gemm":
         rank = int(os.environ.get("RANK", "0"))
         if rank == 0:

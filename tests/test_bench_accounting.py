@@ -62,3 +62,26 @@ def test_oracle_pool_runs_one_sequence_per_process():
     assert len(times) == 3 and all(t > 0 for t in times)
     rate, done, el = bench.run_oracle_pool(cfg, 0, 2, budget_s=0.2)
     assert done >= 2 and rate > 0 and el >= 0.2
+
+
+def test_dram_reader_counts_its_bytes_and_stops():
+    """The host-DRAM load of `--config host_contention`: a spawned reader adds one buffer's
+    bytes per pass to the shared counter and exits once told to stop."""
+    import multiprocessing as mp
+    import time
+    ctx = mp.get_context("spawn")
+    stop, counter, ready = ctx.Event(), ctx.Value("d", 0.0), ctx.Queue()
+    nbytes = 8 << 20
+    p = ctx.Process(target=bench._dram_reader, args=(nbytes, stop, counter, ready), daemon=True)
+    p.start()
+    try:
+        ready.get(timeout=120)
+        t_end = time.time() + 60
+        while counter.value < 3 * nbytes and time.time() < t_end:
+            time.sleep(0.05)
+        assert counter.value >= 3 * nbytes
+        assert counter.value % nbytes == 0
+    finally:
+        stop.set()
+        p.join(timeout=30)
+    assert p.exitcode == 0
