@@ -423,9 +423,10 @@ int launch_projection(const ProjArgs& a, cudaStream_t st) {
   }
   const int tiles = a.Hkv * p.nt;
   // each cluster splits one tile's reduction dimension; about 240 CTAs in total (one wave
-  // at two CTAs per SM) measured best on B200: clusters of 5 for the 8B-shaped layer (48
-  // tiles, 16.9 us vs 18.0 at 4 and 21.0 at 3) and of 3 for the 70B-shaped one (80 tiles,
-  // 41.6 us vs 45.6 at 2 and 51.5 at 5)
+  // at two CTAs per SM) measured best on B200 (launches back to back, W read from HBM):
+  // clusters of 5 for the 8B-shaped layer (48 tiles, 16.4 us vs 16.6 at 4, 16.7 at 3 and
+  // 22.5 at 6; with W in L2 12.3 vs 14.3 and 16.4) and of 3 for the 70B-shaped one (80
+  // tiles, 36.0 us vs 39.5 at 2 and 45.4 at 4)
   int CS = a.cluster > 0 ? a.cluster : (240 + tiles / 2) / tiles;
   if (CS < 1) CS = 1;
   if (CS > 8) CS = 8;
