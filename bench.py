@@ -1007,6 +1007,29 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
         _nvtx_end()
         per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(steps)]
 
+        # ---- launch A/B under the same sustained load: interleaved blocks of back-to-back
+        # steps with the two kernels overlapped (programmatic dependent launch, the default)
+        # and launched serially, no events inside a block
+        _nvtx("launch A/B " + cfg.name)
+        n_ab = steps if wl.kv_host_bytes == 0 else min(steps, 5)
+        ab = {0: [], 1: []}
+        for _ in range(2):
+            for mode in (0, 1):
+                wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant, serial_launch=mode)
+                wl.step()
+                barrier()
+                a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a0.record()
+                for _ in range(n_ab):
+                    wl.step()
+                a1.record()
+                barrier()
+                ab[mode].append(a0.elapsed_time(a1) / n_ab)
+        wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant)
+        ab_ms = [sum(ab[0]) / len(ab[0]), sum(ab[1]) / len(ab[1])]
+        pass_mhz["launch_ab"] = sm_clock_now(local)
+        _nvtx_end()
+
         # ---- per-stage durations: the same steps launched serially (no programmatic
         # dependent launch, so each kernel runs alone), with events between the two launches
         _nvtx("stages " + cfg.name)
@@ -1048,9 +1071,10 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
 
         # ---- max over ranks
         p10, p50, p90 = percentiles(per_step)
-        vals = reduce_max_over_ranks([t_ms, e2e_ms, p10, p50, p90, proj_b2b_ms] + stage_ms, dist, dev)
+        vals = reduce_max_over_ranks([t_ms, e2e_ms, p10, p50, p90, proj_b2b_ms] + ab_ms + stage_ms, dist, dev)
         t_ms, e2e_ms, p10, p50, p90, proj_b2b_ms = vals[:6]
-        stage_ms = vals[6:]
+        ab_ms = vals[6:8]
+        stage_ms = vals[8:]
         ms = t_ms / steps
         value = replica_throughput(cfg.B, world, ms)
 
@@ -1085,6 +1109,11 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
                          "project_back_to_back": proj_b2b_ms,
                          "project_back_to_back_timing": "%d serial launches queued behind a sleep kernel, "
                                                         "between two events, W from HBM" % n_proj},
+            "launch_ab": {"overlapped_ms_per_step": ab_ms[0], "serial_ms_per_step": ab_ms[1],
+                          "steps_per_block": n_ab, "blocks_per_mode": 2,
+                          "timing": "interleaved blocks of back-to-back steps, no events inside a block: "
+                                    "the default launch (the two kernels overlapped by programmatic "
+                                    "dependent launch) against serial launches under the same load"},
             "projection_roofline": {"bound": "hbm", "kernel": "proj_umma_kernel",
                                     "achieved": wl.w_bytes / (proj_b2b_ms * 1e-3) / 1e9, "peak": peak,
                                     "unit": "GB/s", "frac": wl.w_bytes / (proj_b2b_ms * 1e-3) / 1e9 / peak,
