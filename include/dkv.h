@@ -83,7 +83,8 @@ typedef struct dkv_pool_config {
 /* Launch tunables; 0 means "choose automatically". */
 typedef struct dkv_tuning {
   int32_t attn_splits;   /* split-K factor of the attention grid (per sequence, kv head) */
-  int32_t proj_splits;   /* cluster size of the projection (its reduction split), <= 16 */
+  int32_t proj_splits;   /* cluster size of the projection (its reduction split), 0..8;
+                            above hidden/64 it is cut to hidden/64 */
   int32_t attn_variant;  /* attention kernel: 0 automatic (see dkv_decode_attn_variant),
                             5 CUDA-core products with q in registers (G <= 4: three
                             one-warp consumer slots, a 6-stage ring, 4 CTAs/SM; G = 8: two

@@ -259,7 +259,7 @@ int dkv_pool_set_tuning(dkv_pool* p, const dkv_tuning* t) {
   if (!p) return set_error(DKV_ERR_ARG, "dkv_pool_set_tuning: null pool");
   if (t) {
     const int v = t->attn_variant;
-    if (t->attn_splits < 0 || t->proj_splits < 0 || t->proj_splits > 16 || (v != 0 && v != 1 && v != 5 && v != 6 && v != 7) ||
+    if (t->attn_splits < 0 || t->proj_splits < 0 || t->proj_splits > 8 || (v != 0 && v != 1 && v != 5 && v != 6 && v != 7) ||
         t->attn_lsu_hbm < 0 || t->attn_lsu_hbm > 3 || t->serial_launch < 0 || t->serial_launch > 3 ||
         t->wait_limit_us < 0 || t->test_withhold_block < 0 || t->test_withhold_block > 1)
       return set_error(DKV_ERR_ARG, "dkv_pool_set_tuning: value out of range");

@@ -190,6 +190,9 @@ def test_argument_errors():
         with pytest.raises(dkv.DkvError):
             dkv.dkv_decode_step(ctx.pool, 0, inp.x.cuda(), inp.W.cuda(), ctx.table, ctx.seq_lens,
                                 ctx.tier_map, cfg.Hq, cfg.theta, out, ws)
+        for bad in (dict(proj_splits=9), dict(proj_splits=-1), dict(attn_splits=-1), dict(attn_variant=2)):
+            with pytest.raises(dkv.DkvError):
+                dkv.dkv_pool_set_tuning(ctx.pool, **bad)
     finally:
         ctx.close()
 
