@@ -88,21 +88,55 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // o over the entries in index order, so the result does not depend on which CTA merges
 // and the fused and the standalone combine produce identical bits. The accumulator loads
 // of four entries for all of a lane's D/32 dims are in flight together.
-template <int D>
+template <int D, int UM, int UA>
 __device__ __forceinline__ void combine_head_warp(const float2* __restrict__ ml, const float* __restrict__ acc,
                                                   int n, int64_t base, int stride, float sn,
                                                   const float* __restrict__ vn, uint16_t* __restrict__ out,
                                                   int lane) {
   constexpr int DL = D / 32;
+  // UM: (m, l) loads a lane has in flight together; UA: splits whose accumulator loads are
+  // in flight together (the caller's register budget sets both). The partial states sit in
+  // L2 (written by the other split CTAs moments ago): every round of loads costs a full L2
+  // round trip, so the loads of a round are issued before any is used. The arithmetic
+  // order is fixed (lane l takes splits l, l + 32, ... in increasing order, then a
+  // butterfly; the accumulators in split order), so the fused and the standalone combine
+  // give identical bits.
   float M = sn;
-  for (int s = lane; s < n; s += 32) M = fmaxf(M, __ldcg(ml + base + (int64_t)s * stride).x);
+  if constexpr (UM == 1) {  // one load at a time (the tightest register budget)
+    for (int s = lane; s < n; s += 32) M = fmaxf(M, __ldcg(ml + base + (int64_t)s * stride).x);
+  } else {
+    for (int s0 = lane; s0 < n; s0 += 32 * UM) {
+      float x[UM];
+#pragma unroll
+      for (int u = 0; u < UM; ++u) {
+        const int s = s0 + 32 * u;
+        x[u] = s < n ? __ldcg(ml + base + (int64_t)s * stride).x : -INFINITY;
+      }
+#pragma unroll
+      for (int u = 0; u < UM; ++u) M = fmaxf(M, x[u]);
+    }
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const float wn = exp2f(sn - M);  // M >= s_new is finite; an empty state (m = -inf) weighs 0
   float Lp = 0.f;
-  for (int s = lane; s < n; s += 32) {
-    const float2 m = __ldcg(ml + base + (int64_t)s * stride);
-    Lp = fmaf(m.y, exp2f(m.x - M), Lp);
+  if constexpr (UM == 1) {
+    for (int s = lane; s < n; s += 32) {
+      const float2 m = __ldcg(ml + base + (int64_t)s * stride);
+      Lp = fmaf(m.y, exp2f(m.x - M), Lp);
+    }
+  } else {
+    for (int s0 = lane; s0 < n; s0 += 32 * UM) {
+      float2 x[UM];
+#pragma unroll
+      for (int u = 0; u < UM; ++u) {
+        const int s = s0 + 32 * u;
+        x[u] = s < n ? __ldcg(ml + base + (int64_t)s * stride) : make_float2(-INFINITY, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < UM; ++u)
+        if (s0 + 32 * u < n) Lp = fmaf(x[u].y, exp2f(x[u].x - M), Lp);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) Lp += __shfl_xor_sync(0xffffffffu, Lp, o);
@@ -115,6 +149,22 @@ __device__ __forceinline__ void combine_head_warp(const float2* __restrict__ ml,
     float wmine = 0.f;
     if (lane < cnt) wmine = exp2f(__ldcg(ml + base + (int64_t)(s0 + lane) * stride).x - M);
     int t = 0;
+    if constexpr (UA > 4) {
+      for (; t + UA <= cnt; t += UA) {
+        float a[UA][DL];
+#pragma unroll
+        for (int u = 0; u < UA; ++u)
+#pragma unroll
+          for (int k = 0; k < DL; ++k)
+            a[u][k] = __ldcg(acc + (base + (int64_t)(s0 + t + u) * stride) * D + lane + 32 * k);
+#pragma unroll
+        for (int u = 0; u < UA; ++u) {
+          const float w = __shfl_sync(0xffffffffu, wmine, t + u);
+#pragma unroll
+          for (int k = 0; k < DL; ++k) A[k] = fmaf(a[u][k], w, A[k]);
+        }
+      }
+    }
     for (; t + 4 <= cnt; t += 4) {
       float a[4][DL];
 #pragma unroll
@@ -220,7 +270,11 @@ __device__ __forceinline__ void attn_merge_combine(const AttnParams& p, uint8_t*
                              (int64_t)gridDim.z * p.Hq))
           continue;
         const float sn = new_token_score(p.qs + ((int64_t)b * p.Hq + hg) * D, kn, D, lane);
-        combine_head_warp<D>(p.part_ml, p.part_acc, p.S, ((int64_t)b * p.Hq + hg) * p.S, 1, sn,
+        // the three-CTAs-per-SM G = 8 shape (two slots of two warps) runs at its full
+        // register budget: its merge keeps one (m, l) load and four splits in flight, the
+        // other shapes eight of each
+        constexpr bool tight = HPW * WPB == 8 && WPB == 2 && SL == 2;
+        combine_head_warp<D, tight ? 1 : 8, tight ? 4 : 8>(p.part_ml, p.part_acc, p.S, ((int64_t)b * p.Hq + hg) * p.S, 1, sn,
                              p.vnew + ((int64_t)b * pool.Hkv + g) * D, p.out + ((int64_t)b * p.Hq + hg) * D, lane);
       }
       if (threadIdx.x == 0) p.cnt[(int64_t)b * pool.Hkv + g] = 0;
@@ -872,7 +926,7 @@ __global__ void __launch_bounds__(32) combine_kernel(int Hq, int Hkv, int S, con
   const int hg = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
   const int g = hg / (Hq / Hkv);
   const float sn = new_token_score(qs + ((int64_t)b * Hq + hg) * D, knew + ((int64_t)b * Hkv + g) * D, D, lane);
-  combine_head_warp<D>(ml, acc, S, ((int64_t)b * Hq + hg) * S, 1, sn, vnew + ((int64_t)b * Hkv + g) * D,
+  combine_head_warp<D, 8, 16>(ml, acc, S, ((int64_t)b * Hq + hg) * S, 1, sn, vnew + ((int64_t)b * Hkv + g) * D,
                        out + ((int64_t)b * Hq + hg) * D, lane);
 }
 
