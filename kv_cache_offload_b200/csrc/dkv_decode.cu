@@ -17,16 +17,27 @@ namespace dkv {
 
 // Automatic split count. Tensor-core kernels: one wave of about 7/8 of the resident CTA
 // slots, at most 32 splits (the last split CTA of each (sequence, kv head) merges all of
-// them). Measured best on B200 for uniform batches of 2 K - 32 K tokens, B = 4..32 (8B
-// shape, B=16 x 32 K: 311 us at 4 splits vs 326 us at 13 = 2.8 waves); more waves only
-// add per-CTA setup and merge work. CUDA-core kernels: about 2.9 waves (their best).
-// Host-bound configurations are insensitive to the split count.
+// them). CUDA-core kernels, measured on B200 (attention alone, all blocks in HBM, B in
+// {1, 2, 4, 8, 16, 32} x {8 K, 32 K} tokens and B in {1, 4} x 128 K, split counts from
+// 0.3 to 3.5 waves of each shape's CTA slots): a grid just under a whole number of waves
+// is fast and one just over it slow (its last CTAs run alone), and fewer, longer splits
+// pay less per-CTA setup and merge work. G = 4: the most splits that fit in one wave up
+// to 64 (sequence, kv head) units, two waves above that (B=16 x 32 K: 334 us at 9 splits
+// vs 349 at 13; B=32 x 32 K: 660 vs 711 at 7; B=1 x 128 K: 102 vs 121 at 161; B=4 x 32 K:
+// 97 vs 114). The one-CTA-per-SM G = 8 shape: one wave (B=1 x 32 K: 66 vs 76 us at 54).
+// The three-CTA G = 8 shape keeps about 2.9 waves (within 1-4% of its best from 2.3 to 2.9
+// waves), as do the group sizes not measured. Host-bound configurations are insensitive.
 static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant) {
   const int slots = pool->num_sms * attention_ctas_per_sm(G, variant);
   const int units = B * Hkv;
   if (variant == 6 || variant == 7) {
     const int s = (7 * slots + 4 * units) / (8 * units);  // round(7/8 * slots / units)
     return s > 32 ? 32 : s;
+  }
+  if (G == 4 || (G == 8 && variant == 1)) {
+    const int waves = (G == 4 && units > 64) ? 2 : 1;
+    const int s = waves * slots / units;  // the most splits that fit in `waves` waves
+    return s < 1 ? 1 : s;
   }
   return (29 * slots + 5 * units) / (10 * units);
 }
@@ -41,7 +52,8 @@ static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant)
 // B=32 x 8 K: 198 vs 205; B=4 x 32 K at 38 blocks: 118 vs 117); G = 8 takes it once its
 // splits keep at least 6 blocks and there are at most 64 of them (B=8 x 32 K: 304 vs 584
 // us; B=32 x 2 K: 100 vs 154; B=8 x 2 K at 6.5 blocks: 49 vs 60; a single sequence, 129-161
-// splits: 55-96 vs 33-84). Other group sizes: variant 1.
+// splits: 55-96 vs 33-84). Other group sizes: variant 1. Re-checked at the split counts of
+// auto_splits above (the same sweep): the G = 4 threshold still picks the faster shape.
 static int resolve_attn_variant(const dkv_pool* pool, int B, int Hkv, int G, int max_blocks) {
   const int v = pool->tuning.attn_variant;
   if (v != 0) return v;
