@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="dkv", choices=["dkv", "reference"])
     ap.add_argument("--config", default="70b_mixed",
-                    choices=sorted(WL.CONFIGS) + ["gemm", "layout", "adaptive", "host_contention"],
+                    choices=sorted(WL.CONFIGS) + ["gemm", "layout", "adaptive", "host_contention", "attn_sweep"],
                     help="decode workload (default: the largest single-GPU configuration; the all-HBM "
                          "8B-shaped layer is then reported beside it as hbm_line)")
     ap.add_argument("--no-hbm-line", action="store_true", help="skip the all-HBM line of the default run")
@@ -875,6 +875,70 @@ def run_host_contention(args):
     print(json.dumps(line), flush=True)
 
 
+def run_attn_sweep(args):
+    """Attention alone (all blocks in HBM, serial launches) over split counts for both
+    CUDA-core shapes, per batch x context, on the 8B-shaped (G = 4) and 70B-shaped (G = 8)
+    layers: split counts at 0.3 to 3.5 waves of each shape's CTA slots (148 SMs x CTAs per
+    SM: G = 4 variant 1 three, variant 5 four; G = 8 variant 1 one, variant 5 three), plus
+    the automatic choice. 15 launches back to back between two events, best of 2 rounds."""
+    import dataclasses
+    import kv_cache_offload_b200 as dkv
+    from kv_cache_offload_b200.build import build
+    build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    per_sm = {(4, 1): 3, (4, 5): 4, (8, 1): 1, (8, 5): 3}
+    waves = (0.3, 0.43, 0.58, 0.72, 0.86, 1.0, 1.15, 1.45, 1.73, 2.0, 2.3, 2.9, 3.5)
+    cases = ([("8b_hbm", B, c) for B in (1, 2, 4, 8, 16, 32) for c in (8192, 32768)]
+             + [("8b_hbm", 1, 131072), ("8b_hbm", 4, 131072)]
+             + [("70b_hbm", B, c) for B in (1, 4, 8, 32) for c in (8192, 32768)] + [("70b_hbm", 1, 131072)])
+    rows = []
+    for name, B, ctx in cases:
+        cfg = dataclasses.replace(WL.CONFIGS[name], B=B, ctx=ctx, ctx_range=None, tier_policy="hbm")
+        wl = Workload(cfg, seed=0)
+        try:
+            lay, units = wl.lay, cfg.B * cfg.Hkv
+            auto = (dkv.dkv_decode_attn_variant(wl.pool, cfg.B, lay.max_blocks, cfg.Hq),
+                    dkv.dkv_decode_attn_splits(wl.pool, cfg.B, lay.max_blocks, cfg.Hq))
+            res = {}
+            for variant in (1, 5):
+                slots = sms * per_sm[(cfg.G, variant)]
+                Ss = {max(1, min(lay.max_blocks, round(w * slots / units))) for w in waves}
+                if auto[0] == variant:
+                    Ss.add(auto[1])
+                for S in sorted(Ss):
+                    wl.set_tuning(attn_splits=S, attn_variant=variant, serial_launch=1)
+                    wl.project()
+                    c = wl.cfg
+                    attend = lambda: dkv.dkv_decode_attend(wl.pool, 0, wl.table, wl.lens, wl.tmap, c.H, c.Hq, wl.ws,
+                                                           out=wl.out)
+                    for _ in range(3):
+                        attend()
+                    best = float("inf")
+                    for _ in range(2):
+                        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        torch.cuda._sleep(3_000_000)  # the host queues the launches meanwhile
+                        a.record()
+                        for _ in range(15):
+                            attend()
+                        b.record()
+                        b.synchronize()
+                        best = min(best, a.elapsed_time(b) * 1e3 / 15)
+                    res[(variant, S)] = best
+            assert dkv.dkv_check(wl.pool) == dkv.DKV_OK, dkv.dkv_last_error()
+            bk = min(res, key=res.get)
+            rows.append({"layer": name, "B": B, "ctx": ctx, "G": cfg.G, "units": units, "blocks": lay.max_blocks,
+                         "kv_bytes": wl.kv_bytes, "auto": [auto[0], auto[1], res[auto]],
+                         "best": [bk[0], bk[1], res[bk]],
+                         "points_us": {"v%d S=%d" % k: v for k, v in sorted(res.items())}})
+        finally:
+            wl.close()
+        torch.cuda.empty_cache()
+    print(json.dumps({"metric": "attention alone (us) over split counts and CUDA-core shapes, all blocks in HBM",
+                      "sms": sms, "rows": rows}), flush=True)
+
+
 def run_adaptive(args):
     """Adaptive placement (hot blocks in HBM, cold blocks read in place from the host tier)
     over a 4-layer slice of the 8B-shaped model, B=16 x 32768 cached tokens (8 GiB of KV),
@@ -1222,6 +1286,8 @@ def main():
         return run_adaptive(args)
     if args.config == "host_contention":
         return run_host_contention(args)
+    if args.config == "attn_sweep":
+        return run_attn_sweep(args)
     if args.config == "gemm":
         rank = int(os.environ.get("RANK", "0"))
         if rank == 0:
