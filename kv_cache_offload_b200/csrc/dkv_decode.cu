@@ -25,8 +25,10 @@ namespace dkv {
 // to 64 (sequence, kv head) units, two waves above that (B=16 x 32 K: 334 us at 9 splits
 // vs 349 at 13; B=32 x 32 K: 660 vs 711 at 7; B=1 x 128 K: 102 vs 121 at 161; B=4 x 32 K:
 // 97 vs 114). The one-CTA-per-SM G = 8 shape: one wave (B=1 x 32 K: 66 vs 76 us at 54).
-// The three-CTA G = 8 shape keeps about 2.9 waves (within 1-4% of its best from 2.3 to 2.9
-// waves), as do the group sizes not measured. Host-bound configurations are insensitive.
+// The three-CTA G = 8 shape: the most splits within 2.33 waves (B=4 x 8 K: 63.0 vs 67.0 us
+// at 2.9 waves; B=32 x 32 K: 1108 vs 1119; B=16 x 32 K: 566 vs 573). Group sizes not
+// measured: about 2.9 waves. Host-bound configurations are insensitive (70B layer with 80%
+// of its blocks in the host tier: 70.75 ms at 4 and 5 splits).
 static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant) {
   const int slots = pool->num_sms * attention_ctas_per_sm(G, variant);
   const int units = B * Hkv;
@@ -37,6 +39,10 @@ static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant)
   if (G == 4 || (G == 8 && variant == 1)) {
     const int waves = (G == 4 && units > 64) ? 2 : 1;
     const int s = waves * slots / units;  // the most splits that fit in `waves` waves
+    return s < 1 ? 1 : s;
+  }
+  if (G == 8) {  // the three-CTA shape: the most splits within 2.33 waves
+    const int s = 233 * slots / (100 * units);
     return s < 1 ? 1 : s;
   }
   return (29 * slots + 5 * units) / (10 * units);
