@@ -282,7 +282,13 @@ int dkv_decode_step_static(dkv_pool* pool, int layer, const uint16_t* x, const u
 /* Size in bytes of the per-device static workspace dkv_decode_step_static uses. */
 size_t dkv_decode_static_workspace_capacity(void);
 
-/* The attention split-K factor dkv_decode_step uses for this shape (after tuning). */
+/* The attention split-K factor dkv_decode_step uses for this shape: the pool's
+ * dkv_tuning.attn_splits, or, when that is 0, the automatic count. With units = B * Hkv
+ * and slots = the GPU's SMs x the chosen kernel shape's CTAs per SM: Hq/Hkv = 4, the most
+ * splits that fit in one wave of slots (two waves above 64 units); Hq/Hkv = 8, one wave
+ * for variant 1 and the most within 2.33 waves for variant 5; other group sizes, about 2.9
+ * waves; the tensor-core variants, about 7/8 of one wave and at most 32. Never more than
+ * max_blocks. Returns the count (> 0) or a negative DKV_ERR_* code. */
 int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 
 /* The attention kernel variant dkv_decode_step runs for this shape: the pool's
