@@ -130,6 +130,36 @@ def test_automatic_attention_variant():
         dkv.dkv_pool_destroy(pool)
 
 
+@pytest.mark.parametrize("Hq", [8, 16, 32, 64])
+def test_automatic_split_count_respects_its_wave_bound(Hq):
+    """Over many batch sizes and table widths (8 kv heads, so G = 1, 2, 4, 8): the automatic
+    split count is at least 1, at most the table width, and its grid fits the documented
+    number of waves of the chosen shape's CTA slots whenever the width allows it."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    per_sm = {(4, 1): 3, (4, 5): 4, (8, 1): 1, (8, 5): 3}
+    pool = dkv.dkv_pool_create(1, 8, 128, 4, 1, block_tokens=16)
+    try:
+        G = Hq // 8
+        for B in (1, 2, 3, 5, 8, 13, 16, 24, 32):
+            for blocks in (1, 2, 7, 33, 130, 513, 2050, 8193):
+                S = dkv.dkv_decode_attn_splits(pool, B, blocks, Hq)
+                v = dkv.dkv_decode_attn_variant(pool, B, blocks, Hq)
+                assert 1 <= S <= blocks, (B, blocks, Hq, S)
+                units = B * 8
+                if G == 4 or (G == 8 and v == 1):
+                    waves = 2 if (G == 4 and units > 64) else 1
+                elif G == 8:
+                    waves = 2.33
+                else:
+                    continue
+                slots = sms * per_sm[(G, v)]
+                assert units * S <= max(units, waves * slots), (B, blocks, Hq, v, S)
+                if S < blocks:  # not capped by the table: the most splits within the bound
+                    assert units * (S + 1) > waves * slots, (B, blocks, Hq, v, S)
+    finally:
+        dkv.dkv_pool_destroy(pool)
+
+
 def test_bad_table_entries_are_flagged_not_fatal():
     cfg = WL.small_config(B=2, ctx_range=(40, 60), host_prob=0.5)
     inp = WL.make_decode_inputs(cfg)
