@@ -291,6 +291,10 @@ class Workload:
         self.dkv.dkv_decode_step(self.pool, 0, self.x, self.next_W(), self.table, self.lens, self.tmap, c.Hq,
                                  c.theta, self.out, self.ws)
 
+    def attend(self):
+        c = self.cfg
+        self.dkv.dkv_decode_attend(self.pool, 0, self.table, self.lens, self.tmap, c.H, c.Hq, self.ws, out=self.out)
+
     def project(self):
         c = self.cfg
         self.dkv.dkv_decode_project(self.pool, 0, self.x, self.next_W(), self.table, self.lens, self.tmap, c.Hq,
@@ -1075,22 +1079,26 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
         # steps with the two kernels overlapped (programmatic dependent launch, the default)
         # and launched serially, no events inside a block
         _nvtx("launch A/B " + cfg.name)
+        # (and blocks of the attention alone, launched the same way: what the overlapped step
+        # costs beyond its attention is the projection's exposed part)
         n_ab = steps if wl.kv_host_bytes == 0 else min(steps, 5)
-        ab = {0: [], 1: []}
+        ab = {0: [], 1: [], 2: []}
         for _ in range(2):
-            for mode in (0, 1):
-                wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant, serial_launch=mode)
-                wl.step()
+            for mode in (0, 1, 2):
+                wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant,
+                              serial_launch=1 if mode == 2 else mode)
+                run = wl.step if mode < 2 else wl.attend
+                run()
                 barrier()
                 a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a0.record()
                 for _ in range(n_ab):
-                    wl.step()
+                    run()
                 a1.record()
                 barrier()
                 ab[mode].append(a0.elapsed_time(a1) / n_ab)
         wl.set_tuning(args.attn_splits, args.proj_splits, attn_variant=args.attn_variant)
-        ab_ms = [sum(ab[0]) / len(ab[0]), sum(ab[1]) / len(ab[1])]
+        ab_ms = [sum(ab[m]) / len(ab[m]) for m in (0, 1, 2)]
         pass_mhz["launch_ab"] = sm_clock_now(local)
         _nvtx_end()
 
@@ -1137,8 +1145,8 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
         p10, p50, p90 = percentiles(per_step)
         vals = reduce_max_over_ranks([t_ms, e2e_ms, p10, p50, p90, proj_b2b_ms] + ab_ms + stage_ms, dist, dev)
         t_ms, e2e_ms, p10, p50, p90, proj_b2b_ms = vals[:6]
-        ab_ms = vals[6:8]
-        stage_ms = vals[8:]
+        ab_ms = vals[6:9]
+        stage_ms = vals[9:]
         ms = t_ms / steps
         value = replica_throughput(cfg.B, world, ms)
 
@@ -1174,10 +1182,12 @@ def decode_line(cfg: WL.DecodeConfig, args, world, rank, local, dist, dev, full:
                          "project_back_to_back_timing": "%d serial launches queued behind a sleep kernel, "
                                                         "between two events, W from HBM" % n_proj},
             "launch_ab": {"overlapped_ms_per_step": ab_ms[0], "serial_ms_per_step": ab_ms[1],
+                          "attention_alone_ms": ab_ms[2], "step_minus_attention_ms": ab_ms[0] - ab_ms[2],
                           "steps_per_block": n_ab, "blocks_per_mode": 2,
                           "timing": "interleaved blocks of back-to-back steps, no events inside a block: "
                                     "the default launch (the two kernels overlapped by programmatic "
-                                    "dependent launch) against serial launches under the same load"},
+                                    "dependent launch) against serial launches and against the attention "
+                                    "launched alone, under the same load"},
             "projection_roofline": {"bound": "hbm", "kernel": "proj_umma_kernel",
                                     "achieved": wl.w_bytes / (proj_b2b_ms * 1e-3) / 1e9, "peak": peak,
                                     "unit": "GB/s", "frac": wl.w_bytes / (proj_b2b_ms * 1e-3) / 1e9 / peak,
