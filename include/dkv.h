@@ -286,7 +286,8 @@ size_t dkv_decode_static_workspace_capacity(void);
  * dkv_tuning.attn_splits, or, when that is 0, the automatic count. With units = B * Hkv
  * and slots = the GPU's SMs x the chosen kernel shape's CTAs per SM: Hq/Hkv = 4, the most
  * splits that fit in one wave of slots (two waves above 64 units); Hq/Hkv = 8, one wave
- * for variant 1 and the most within 2.33 waves for variant 5; other group sizes, about 2.9
+ * for variant 1 and the most within 2.33 waves for variant 5 (0.86 of a wave where that
+ * would be more than 64 splits); other group sizes, about 2.9
  * waves; the tensor-core variants, about 7/8 of one wave and at most 32. Never more than
  * max_blocks. Returns the count (> 0) or a negative DKV_ERR_* code. */
 int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
@@ -294,7 +295,8 @@ int dkv_decode_attn_splits(const dkv_pool* pool, int B, int max_blocks, int num_
 /* The attention kernel variant dkv_decode_step runs for this shape: the pool's
  * dkv_tuning.attn_variant, or, when that is 0, the automatic choice (Hq/Hkv = 4: 5 when its
  * split-K ranges keep at least 39 blocks of the table each, else 1; Hq/Hkv = 8: 5 when they
- * keep at least 6 blocks and there are at most 64 of them, else 1; other group sizes: 1).
+ * keep at least 6 blocks and there are at most 64 of them (at least 40 blocks when the
+ * automatic count was cut under one wave), else 1; other group sizes: 1).
  * Returns the variant (> 0) or a negative DKV_ERR_* code. */
 int dkv_decode_attn_variant(const dkv_pool* pool, int B, int max_blocks, int num_q_heads);
 

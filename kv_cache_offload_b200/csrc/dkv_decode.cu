@@ -41,8 +41,10 @@ static int auto_splits(const dkv_pool* pool, int B, int Hkv, int G, int variant)
     const int s = waves * slots / units;  // the most splits that fit in `waves` waves
     return s < 1 ? 1 : s;
   }
-  if (G == 8) {  // the three-CTA shape: the most splits within 2.33 waves
-    const int s = 233 * slots / (100 * units);
+  if (G == 8) {  // the three-CTA shape: the most splits within 2.33 waves, or, where that
+                 // would be more than 64 (a single sequence), within 0.86 of a wave
+    int s = 233 * slots / (100 * units);
+    if (s > 64) s = 86 * slots / (100 * units);
     return s < 1 ? 1 : s;
   }
   return (29 * slots + 5 * units) / (10 * units);
@@ -68,6 +70,11 @@ static int resolve_attn_variant(const dkv_pool* pool, int B, int Hkv, int G, int
   if (s5 < 1) s5 = 1;
   const int blocks_per_split = max_blocks / s5;
   if (G == 4) return blocks_per_split >= 39 ? 5 : 1;
+  // G = 8 and a single sequence (automatic splits cut to under one wave): the three-CTA
+  // shape only once its splits keep >= 40 blocks (70B layer, B=1: 128 K tokens 185 vs 230
+  // us, 32 K 64 vs 66, 8 K 33 vs 25)
+  const int slots5 = pool->num_sms * attention_ctas_per_sm(G, 5);
+  if (pool->tuning.attn_splits <= 0 && 233 * slots5 / (100 * B * Hkv) > 64) return blocks_per_split >= 40 ? 5 : 1;
   return blocks_per_split >= 6 && s5 <= 64 ? 5 : 1;
 }
 

@@ -104,10 +104,11 @@ def test_step_is_repeatable():
 def test_automatic_attention_variant():
     """The automatic shape and split count (148 SMs). Splits: G = 4 and the one-CTA G = 8
     shape take the most that fit in one wave of CTA slots (two for G = 4 above 64
-    (sequence, kv head) units), the three-CTA G = 8 shape the most within 2.33 waves, other
-    group sizes about 2.9 waves. Shape: variant 5 for G = 4 while its splits keep >= 39 table blocks each, for
-    G = 8 while they keep >= 6 and number at most 64, else (and for other group sizes)
-    variant 1; an explicit tuning value is taken as is."""
+    (sequence, kv head) units), the three-CTA G = 8 shape the most within 2.33 waves (0.86
+    of a wave where that would exceed 64 splits), other group sizes about 2.9 waves. Shape:
+    variant 5 for G = 4 while its splits keep >= 39 table blocks each, for G = 8 while they
+    keep >= 6 and number at most 64 (>= 40 blocks when cut under a wave), else (and for
+    other group sizes) variant 1; an explicit tuning value is taken as is."""
     pool = dkv.dkv_pool_create(1, 8, 128, 4, 1, block_tokens=16)
     try:
         assert dkv.dkv_decode_attn_variant(pool, 16, 2050, 32) == 5
@@ -121,8 +122,10 @@ def test_automatic_attention_variant():
         assert dkv.dkv_decode_attn_splits(pool, 16, 2050, 64) == 8     # within 2.33 waves of 444
         assert dkv.dkv_decode_attn_variant(pool, 8, 130, 64) == 5      # G = 8: 20 splits of 6
         assert dkv.dkv_decode_attn_variant(pool, 4, 130, 64) == 1      # G = 8: 40 splits of 3
-        assert dkv.dkv_decode_attn_variant(pool, 1, 2050, 64) == 1     # G = 8: 161 splits
-        assert dkv.dkv_decode_attn_splits(pool, 1, 2050, 64) == 18     # one wave of 148 slots
+        assert dkv.dkv_decode_attn_variant(pool, 1, 2050, 64) == 5     # G = 8, one sequence:
+        assert dkv.dkv_decode_attn_splits(pool, 1, 2050, 64) == 47     # 0.86 wave, 43 blocks each
+        assert dkv.dkv_decode_attn_variant(pool, 1, 513, 64) == 1      # 10 blocks per split: the
+        assert dkv.dkv_decode_attn_splits(pool, 1, 513, 64) == 18      # one-CTA shape, one wave
         assert dkv.dkv_decode_attn_variant(pool, 16, 2050, 16) == 1    # G = 2: not measured
         dkv.dkv_pool_set_tuning(pool, attn_variant=7)
         assert dkv.dkv_decode_attn_variant(pool, 16, 2050, 32) == 7
@@ -146,13 +149,13 @@ def test_automatic_split_count_respects_its_wave_bound(Hq):
                 v = dkv.dkv_decode_attn_variant(pool, B, blocks, Hq)
                 assert 1 <= S <= blocks, (B, blocks, Hq, S)
                 units = B * 8
-                if G == 4 or (G == 8 and v == 1):
-                    waves = 2 if (G == 4 and units > 64) else 1
-                elif G == 8:
-                    waves = 2.33
-                else:
+                if G not in (4, 8):
                     continue
                 slots = sms * per_sm[(G, v)]
+                if G == 4 or v == 1:
+                    waves = 2 if (G == 4 and units > 64) else 1
+                else:
+                    waves = 2.33 if 233 * slots // (100 * units) <= 64 else 0.86
                 assert units * S <= max(units, waves * slots), (B, blocks, Hq, v, S)
                 if S < blocks:  # not capped by the table: the most splits within the bound
                     assert units * (S + 1) > waves * slots, (B, blocks, Hq, v, S)
