@@ -589,6 +589,7 @@ def gemm_line(args, rank, dev, steps=None, warmup=None):
     h2d = measure_h2d_peak(dev)
     hb.close()
     ca = res["CPU_AWARE"]["ms"]
+    cpu = gemm_cpu_baseline(A, Btd, M, N, K) if rank == 0 else None
     del A, Btd, C
     line = {"metric": "zero-copy GEMM 10240^3 time (CPU-aware tiling)", "value": ca, "unit": "ms",
             "higher_is_better": False, "n_gpus": 1, "steps": steps, "warmup": warmup,
@@ -602,7 +603,28 @@ def gemm_line(args, rank, dev, steps=None, warmup=None):
                           "naive_model_host_bytes_BM128": (M // 128) * b_bytes,
                           "link": "PCIe (not NVLink-C2C)"},
             "pages_context": {"swap_ms": 65, "naive_ms": 1122, "hardware": "PCIe platform, GPU unstated"}}
+    if cpu:
+        line["cpu_baseline"] = cpu
     return line
+
+
+def gemm_cpu_baseline(A, Btd, M, N, K, n_samples=4096, seed=0):
+    """The oracle's fp64 GEMM entries (one dot product of length K per entry), timed on one
+    host thread for a seeded sample of entries and extrapolated, labelled as such, to all
+    M x N entries of the GEMM."""
+    import numpy as np
+    from oracle import dkv_oracle as O
+    A_bits = A.view(torch.int16).cpu().numpy().view(np.uint16)
+    Bt_bits = Btd.view(torch.int16).cpu().numpy().view(np.uint16)
+    rng = np.random.default_rng(seed)
+    rows, cols = rng.integers(0, M, n_samples), rng.integers(0, N, n_samples)
+    t0 = time.perf_counter()
+    O.gemm_entries(A_bits, Bt_bits, rows, cols)
+    t = time.perf_counter() - t0
+    return {"value": t * (M * N / n_samples) * 1e3, "unit": "ms", "cores": 1, "kind": "oracle",
+            "sample": "%d seeded entries of C in fp64 on one host thread (%.2f s); value = that time "
+                      "extrapolated to all %d x %d entries" % (n_samples, t, M, N),
+            "sample_s": t}
 
 
 def run_layout(args):

@@ -85,3 +85,14 @@ def test_dram_reader_counts_its_bytes_and_stops():
         stop.set()
         p.join(timeout=30)
     assert p.exitcode == 0
+
+
+def test_gemm_cpu_baseline_extrapolates_its_sample():
+    """The GEMM line's CPU baseline: the oracle's fp64 entries timed for a seeded sample on
+    one thread, extrapolated by the ratio of all entries to the sample."""
+    import torch
+    A = (torch.rand((64, 32)) * 2 - 1).to(torch.bfloat16)
+    B = (torch.rand((48, 32)) * 2 - 1).to(torch.bfloat16)
+    r = bench.gemm_cpu_baseline(A, B, 64, 48, 32, n_samples=128)
+    assert r["kind"] == "oracle" and r["cores"] == 1 and r["unit"] == "ms"
+    assert r["value"] == pytest.approx(r["sample_s"] * (64 * 48 / 128) * 1e3)
